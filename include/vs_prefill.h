@@ -1,0 +1,186 @@
+/*
+ * vs_prefill.h -- C ABI of libvs, vertical-slash sparse prefill attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (VSPrefill summary pages, "VSPrefill: Vertical-Slash Sparse
+ * Attention with Lightweight Indexing for Long-Context Prefilling"):
+ *   - attention in long-context prefill concentrates on vertical lines (key
+ *     columns that every later query attends to) and slash lines (diagonals at
+ *     a fixed relative offset o = i - j)  -- Technical Summary, section 2,
+ *     "Core Concept: Vertical-Slash Pattern";
+ *   - a light indexer predicts one score per column and one per offset from
+ *     concat(K with RoPE, V)  -- section 2, "VSIndexer";
+ *   - a cumulative threshold on those scores picks the budgets (k_v, k_s)
+ *     -- section 2, "Adaptive Inference Pipeline", "Dynamic Budgeting";
+ *   - a fused FlashAttention-style kernel attends each query to the union of
+ *     the selected columns and the keys at the selected offsets behind it,
+ *     without a precomputed mask -- section 2, "Fused Kernel Execution".
+ *
+ * Conventions for every call:
+ *   - Every pointer argument is a DEVICE pointer on the current CUDA device
+ *     (except `flags` of vs_read_device_status); the caller owns every buffer (inputs,
+ *     outputs, workspace) and the stream.  The library allocates nothing,
+ *     keeps no mutable global state, never writes its inputs and overwrites
+ *     its outputs completely.
+ *   - Calls are asynchronous on `stream`; selected counts stay on the device,
+ *     so select -> attention needs no host synchronisation.
+ *   - Host-side argument checks run before anything is launched and return
+ *     VS_ERR_INVALID_ARG / VS_ERR_UNSUPPORTED / VS_ERR_WORKSPACE.  A failed
+ *     launch returns VS_ERR_CUDA.  Device-side problems (an index outside
+ *     [0, N), a count above its row length, a bounded wait that gave up) are
+ *     OR-ed into a status word at the start of the workspace; read it with
+ *     vs_read_device_status.  Kernels never trap, assert or print.
+ *   - Tensors are token-major: element (t, h, c) of Q lives at
+ *     Q[t * q_stride_tok + h * d + c]; K and V likewise with kv_stride_tok.
+ *     Strides are in elements and must be multiples of 8 (16-byte rows).
+ *   - GQA: query head h reads KV head h / (Hq / Hkv) and index-set head
+ *     h * H_sel / Hq.
+ */
+#ifndef VS_PREFILL_H
+#define VS_PREFILL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VS_OK = 0,
+  VS_ERR_INVALID_ARG = 1,    /* null pointer, bad size, k/cap/tau out of range */
+  VS_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. d not in {64,128}) */
+  VS_ERR_WORKSPACE = 3,      /* workspace missing, misaligned or too small */
+  VS_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  VS_ERR_DEVICE_TIMEOUT = 5, /* returned by vs_read_device_status */
+  VS_ERR_DEVICE_BOUNDS = 6   /* returned by vs_read_device_status */
+} vs_status;
+
+typedef enum { VS_SELECT_TOPK = 0, VS_SELECT_THRESHOLD = 1 } vs_select_mode;
+
+typedef enum { VS_BF16 = 0, VS_FP32 = 1 } vs_dtype;
+
+/* Device status bits (vs_read_device_status `flags`). */
+#define VS_DEVFLAG_TIMEOUT 0x1
+#define VS_DEVFLAG_BOUNDS 0x2
+
+/* Static, human-readable name of a status code. */
+const char* vs_status_string(vs_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int vs_version(void);
+
+/*
+ * vs_index_scores -- the indexer: a shared-weight two-layer linear map on
+ * concat(K with RoPE, V) producing a vertical and a slash score per position
+ * (Technical Summary, section 2, "VSIndexer": input concatenated K and V with
+ * RoPE on K, a bilayer linear network with separate down-projection heads for
+ * the vertical and slash scores, linear cost in n).  The pages do not fix the
+ * exact form; this library reads it as
+ *     x = [k_t ; v_t] (2d values, k first),  h = ReLU(W1 x),
+ *     logits_v[g][t] = W2[0] . h,  logits_s[g][t] = W2[1] . h,
+ * no biases, one weight set shared by all KV heads g.  logits_s[g][t] is the
+ * score of slash offset o = t.
+ *   K, V      [N, Hkv, d] in `dtype` (VS_BF16 or VS_FP32), token stride
+ *             `stride_tok`, head stride `stride_head` (elements).
+ *   W1        fp32 [hidden][2d] row-major (device).   W2  fp32 [2][hidden].
+ *   hidden    1..1024.
+ *   logits_v, logits_s   fp32 [Hkv][N] outputs (device).
+ * Computes in fp32 with fp32 accumulation.
+ */
+vs_status vs_index_scores(const void* K, const void* V, vs_dtype dtype, int N, int Hkv, int d,
+                          int64_t stride_tok, int64_t stride_head, const float* W1,
+                          const float* W2, int hidden, float* logits_v, float* logits_s,
+                          cudaStream_t stream);
+
+/*
+ * vs_select -- per-head budget selection over a score vector (Technical
+ * Summary, section 2, "Dynamic Budgeting": a cumulative-threshold strategy
+ * sets the budgets from the predicted importance scores; the German page's
+ * Inferenz-Pipeline adds the top-k reading).  One call handles H heads.
+ *   scores   fp32 [H][ld_scores] (device), the first N entries of each row used.
+ *            Scores are logits: the "mass" of entry r is softmax(scores)_r.
+ *   Order    score descending, NaN after -inf, ties to the smaller index.
+ *   TOPK     keeps the first k_or_cap entries in that order.
+ *   THRESHOLD keeps the smallest prefix in that order whose mass reaches
+ *            tau (0 < tau <= 1): p_r = exp(s_r - s_max) in fp64, k is the
+ *            smallest k >= 1 with sum_{r<k} p_r >= tau * sum_r p_r; tau = 1
+ *            keeps every entry with p_r > 0; then k = min(k, k_or_cap).
+ *   idx      int32 [H][ld_idx] (device): for each head the kept indices in
+ *            ascending order, then -1 up to k_or_cap (entries past k_or_cap
+ *            untouched).  ld_idx >= k_or_cap.
+ *   count    int32 [H] (device): kept entries per head.
+ *   ws       device workspace of at least vs_select_workspace_size(H, N)
+ *            bytes, 256-byte aligned (holds the device status word).
+ * Requires 1 <= k_or_cap <= N <= 2^20.
+ */
+size_t vs_select_workspace_size(int H, int N);
+vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_select_mode mode,
+                    int k_or_cap, double tau, int32_t* idx, int64_t ld_idx, int32_t* count,
+                    void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * vs_sparse_attn_fwd -- causal vertical-slash sparse attention forward
+ * (Technical Summary, section 2, "Fused Kernel Execution": the vertical and
+ * slash index lists are merged on the fly inside a FlashAttention-style
+ * kernel, with no precomputed mask).  For query i of query head h:
+ *     K_i = { j in V : j <= i }  union  { i - o : o in S, o <= i }
+ * (each key once), and O_i = softmax_j(scale * q_i . k_j) over K_i times V;
+ * LSE_i = log sum_{j in K_i} exp(scale * q_i . k_j).  An empty K_i gives
+ * O_i = 0 and LSE_i = -inf.
+ *   Q        [N, Hq, d], K, V [N, Hkv, d], `dtype` (VS_BF16: tensor-core path;
+ *            VS_FP32: fp32 CUDA-core path).  d in {64, 128}.  Hq % Hkv == 0.
+ *            1 <= N <= 2^22 (dense: 2^24).
+ *   softmax_scale   0 selects 1/sqrt(d).
+ *   H_sel    number of index sets; Hq % H_sel == 0.
+ *   v_idx    int32 [H_sel][v_ld] vertical columns, v_cnt int32 [H_sel];
+ *   s_idx    int32 [H_sel][s_ld] slash offsets,   s_cnt int32 [H_sel]
+ *            (device; as produced by vs_select: entries in [0, N), the first
+ *            cnt entries of each row used; duplicates and order do not matter).
+ *   O        [N, Hq, d] in `dtype` with token stride q_stride_tok (output).
+ *   lse      fp32 [Hq][N] (output) or NULL.
+ *   ws       device workspace, >= vs_attn_workspace_size(N, Hq, H_sel, d)
+ *            bytes, 256-byte aligned.
+ */
+size_t vs_attn_workspace_size(int N, int Hq, int H_sel, int d);
+vs_status vs_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
+                             int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                             float softmax_scale, int H_sel, const int32_t* v_idx, int64_t v_ld,
+                             const int32_t* v_cnt, const int32_t* s_idx, int64_t s_ld,
+                             const int32_t* s_cnt, void* O, float* lse, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * vs_dense_attn_fwd -- dense causal attention with the same kernel
+ * machinery: the "full attention" the pages measure their speed-ups against
+ * (Technical Summary, section 4, Speedup).  Same arguments as
+ * vs_sparse_attn_fwd without the index sets; K_i = [0, i].
+ */
+vs_status vs_dense_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
+                            int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                            float softmax_scale, void* O, float* lse, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/*
+ * Device status of the last call that used `ws`: synchronises `stream`,
+ * copies the status word to `*flags` (VS_DEVFLAG_* bits) and returns VS_OK,
+ * VS_ERR_DEVICE_TIMEOUT or VS_ERR_DEVICE_BOUNDS accordingly.
+ */
+vs_status vs_read_device_status(const void* ws, cudaStream_t stream, int* flags);
+
+/*
+ * Self-test of the device-side wait limit: launches one CTA that waits on an
+ * mbarrier nothing will ever arrive at, through the same bounded-wait code the
+ * kernels use, giving up after `limit_ns` nanoseconds (1e3..1e10).  Afterwards
+ * vs_read_device_status(ws) reports VS_ERR_DEVICE_TIMEOUT.  The CUDA context
+ * stays usable.  `ws` needs 256 bytes.
+ */
+vs_status vs_selftest_wait_timeout(void* ws, uint64_t limit_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VS_PREFILL_H */

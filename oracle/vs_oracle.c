@@ -59,8 +59,9 @@ static double load_elem(const void* base, int dtype, int64_t off) {
  * entry with p_r > 0; Z == 0 gives k = 1; then k = min(k, cap).
  * Output: the k indices in ascending order, padded with -1 up to k_or_cap.
  * `margin` receives min(|prefix(k-1) - tau Z|, |prefix(k) - tau Z|) / Z for
- * the uncapped threshold decision (+inf for TOPK), so callers can flag heads
- * whose decision sits within rounding of the boundary.
+ * the threshold decision (+inf for TOPK, and +inf when the uncapped k exceeds
+ * the cap, since then a +-1 change of k does not change the output), so
+ * callers can flag heads whose output sits within rounding of a boundary.
  */
 typedef struct {
   float s;
@@ -130,6 +131,8 @@ int or_select(const float* s, int N, int mode, int k_or_cap, double tau, int32_t
       *margin = m1 < m2 ? m1 : m2;
     }
     free(p);
+    /* a +-1 change of an uncapped k above the cap leaves min(k, cap) unchanged */
+    if (k > k_or_cap) *margin = INFINITY;
     if (k > k_or_cap) k = k_or_cap;
   }
   for (int r = 0; r < k; ++r) idx[r] = v[r].i;

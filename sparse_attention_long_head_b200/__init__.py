@@ -1,0 +1,217 @@
+"""Python binding of libvs (vertical-slash sparse prefill attention, sm_100a).
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libvs.so``; this module passes device pointers, sizes and the current
+torch CUDA stream to the C ABI declared in ``include/vs_prefill.h`` and turns
+non-OK status codes into ``VsError``.  There is no CPU fallback: if the
+library has not been built, importing the binding's functions raises.
+
+Names follow the C ABI (``vs_select``, ``vs_sparse_attn_fwd``, ...).  Tensors
+are torch CUDA tensors; layouts are those of the header (token-major
+``[N, H, d]`` activations, ``[H, ld]`` index rows).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvs.so")
+
+VS_OK = 0
+VS_ERR_INVALID_ARG = 1
+VS_ERR_UNSUPPORTED = 2
+VS_ERR_WORKSPACE = 3
+VS_ERR_CUDA = 4
+VS_ERR_DEVICE_TIMEOUT = 5
+VS_ERR_DEVICE_BOUNDS = 6
+
+VS_SELECT_TOPK = 0
+VS_SELECT_THRESHOLD = 1
+VS_BF16 = 0
+VS_FP32 = 1
+
+VS_DEVFLAG_TIMEOUT = 0x1
+VS_DEVFLAG_BOUNDS = 0x2
+
+EXPORTS = (
+    "vs_status_string", "vs_version", "vs_index_scores", "vs_select_workspace_size", "vs_select",
+    "vs_attn_workspace_size", "vs_sparse_attn_fwd", "vs_dense_attn_fwd", "vs_read_device_status",
+    "vs_selftest_wait_timeout",
+)
+
+
+class VsError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libvs.so.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libvs.so not built at {LIB_PATH}; run "
+                              "`python -m sparse_attention_long_head_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, U64, D, F = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                                ctypes.c_double, ctypes.c_float)
+        Z = ctypes.c_size_t
+        L.vs_status_string.argtypes = [I]
+        L.vs_status_string.restype = ctypes.c_char_p
+        L.vs_version.argtypes = []
+        L.vs_version.restype = I
+        L.vs_index_scores.argtypes = [P, P, I, I, I, I, I64, I64, P, P, I, P, P, P]
+        L.vs_index_scores.restype = I
+        L.vs_select_workspace_size.argtypes = [I, I]
+        L.vs_select_workspace_size.restype = Z
+        L.vs_select.argtypes = [P, I, I, I64, I, I, D, P, I64, P, P, Z, P]
+        L.vs_select.restype = I
+        L.vs_attn_workspace_size.argtypes = [I, I, I, I]
+        L.vs_attn_workspace_size.restype = Z
+        L.vs_sparse_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, I, P, I64, P, P, I64,
+                                         P, P, P, P, Z, P]
+        L.vs_sparse_attn_fwd.restype = I
+        L.vs_dense_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, P, P, P, Z, P]
+        L.vs_dense_attn_fwd.restype = I
+        L.vs_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
+        L.vs_read_device_status.restype = I
+        L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
+        L.vs_selftest_wait_timeout.restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().vs_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != VS_OK:
+        raise VsError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return VS_BF16
+    if t.dtype == torch.float32:
+        return VS_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------ ABI
+
+
+def vs_version() -> int:
+    return lib().vs_version()
+
+
+def vs_select_workspace_size(H: int, N: int) -> int:
+    return lib().vs_select_workspace_size(H, N)
+
+
+def vs_attn_workspace_size(N: int, Hq: int, H_sel: int, d: int) -> int:
+    return lib().vs_attn_workspace_size(N, Hq, H_sel, d)
+
+
+def vs_index_scores(K, V, W1, W2, logits_v, logits_s, stream=None):
+    """K, V [N, Hkv, d] (bf16 or fp32, head stride = d); W1 [hidden, 2d], W2 [2, hidden]
+    fp32; writes logits_v / logits_s fp32 [Hkv, N]."""
+    N, Hkv, d = K.shape
+    _check(lib().vs_index_scores(_ptr(K), _ptr(V), _dtype(K), N, Hkv, d, K.stride(0), K.stride(1),
+                                 _ptr(W1), _ptr(W2), W1.shape[0], _ptr(logits_v), _ptr(logits_s),
+                                 _stream(stream)), "vs_index_scores")
+
+
+def vs_select(scores, mode, k_or_cap, tau, idx, count, ws, stream=None):
+    """scores fp32 [H, ld >= N] (N = scores.shape[1]); idx int32 [H, ld_idx >= k_or_cap];
+    count int32 [H]; ws from vs_select_workspace_size."""
+    H, N = scores.shape
+    _check(lib().vs_select(_ptr(scores), H, N, scores.stride(0), int(mode), int(k_or_cap),
+                           float(tau), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws), ws.numel(),
+                           _stream(stream)), "vs_select")
+
+
+def vs_sparse_attn_fwd(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, O, lse, ws, softmax_scale=0.0,
+                       stream=None):
+    """Q [N, Hq, d], K/V [N, Hkv, d], O like Q; index rows [H_sel, ld]; lse fp32 [Hq, N] or None."""
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    _check(lib().vs_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype(Q), N, Hq, Hkv, d,
+                                    Q.stride(0), K.stride(0), float(softmax_scale), v_idx.shape[0],
+                                    _ptr(v_idx), v_idx.stride(0), _ptr(v_cnt), _ptr(s_idx),
+                                    s_idx.stride(0), _ptr(s_cnt), _ptr(O), _ptr(lse), _ptr(ws),
+                                    ws.numel(), _stream(stream)), "vs_sparse_attn_fwd")
+
+
+def vs_dense_attn_fwd(Q, K, V, O, lse, ws, softmax_scale=0.0, stream=None):
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    _check(lib().vs_dense_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype(Q), N, Hq, Hkv, d,
+                                   Q.stride(0), K.stride(0), float(softmax_scale), _ptr(O),
+                                   _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "vs_dense_attn_fwd")
+
+
+def vs_read_device_status(ws, stream=None) -> tuple[int, int]:
+    """(status code, flags) of the last call that used ``ws`` (synchronises the stream)."""
+    flags = ctypes.c_int(0)
+    rc = lib().vs_read_device_status(_ptr(ws), _stream(stream), ctypes.byref(flags))
+    return rc, flags.value
+
+
+def vs_selftest_wait_timeout(ws, limit_ns: int, stream=None):
+    _check(lib().vs_selftest_wait_timeout(_ptr(ws), int(limit_ns), _stream(stream)),
+           "vs_selftest_wait_timeout")
+
+
+# ------------------------------------------------------- allocation helpers
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte aligned uint8 device buffer (torch's allocator aligns to 512)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def select(scores, mode, k_or_cap, tau=1.0, ws=None, stream=None):
+    """Allocates outputs and runs vs_select -> (idx [H, k_or_cap], count [H])."""
+    H, N = scores.shape
+    idx = torch.empty((H, k_or_cap), dtype=torch.int32, device=scores.device)
+    cnt = torch.empty(H, dtype=torch.int32, device=scores.device)
+    ws = workspace(vs_select_workspace_size(H, N), scores.device) if ws is None else ws
+    vs_select(scores, mode, k_or_cap, tau, idx, cnt, ws, stream)
+    return idx, cnt
+
+
+def sparse_attention(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, ws=None, with_lse=True, stream=None):
+    N, Hq, d = Q.shape
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, N), dtype=torch.float32, device=Q.device) if with_lse else None
+    if ws is None:
+        ws = workspace(vs_attn_workspace_size(N, Hq, v_idx.shape[0], d), Q.device)
+    vs_sparse_attn_fwd(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, O, lse, ws, stream=stream)
+    return O, lse
+
+
+def dense_attention(Q, K, V, ws=None, with_lse=True, stream=None):
+    N, Hq, d = Q.shape
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, N), dtype=torch.float32, device=Q.device) if with_lse else None
+    ws = workspace(256, Q.device) if ws is None else ws
+    vs_dense_attn_fwd(Q, K, V, O, lse, ws, stream=stream)
+    return O, lse

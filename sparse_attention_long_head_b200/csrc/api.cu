@@ -1,0 +1,228 @@
+// C ABI of libvs: argument validation, workspace layout and launches.
+// Declarations and their documentation: include/vs_prefill.h.
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vs {
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 1;
+  return n > 0 ? n : 1;
+}
+
+// One CTA waits on an mbarrier that nothing arrives at, with the same bounded
+// wait the kernels use; the timeout is recorded in the status word.
+__global__ void wait_selftest_kernel(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtx w{limit_ns, status, &abort_flag};
+  mbar_wait(smem_u32(&bar), 0, w);
+  __syncthreads();
+}
+
+cudaError_t launch_wait_selftest(int* status, uint64_t limit_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+static bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+static vs_status check_attn_common(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                   int N, int Hq, int Hkv, int d, int64_t qs, int64_t kvs,
+                                   float scale, const void* O) {
+  if (!Q || !K || !V || !O) return VS_ERR_INVALID_ARG;
+  if (dtype != VS_BF16 && dtype != VS_FP32) return VS_ERR_INVALID_ARG;
+  if (N < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return VS_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return VS_ERR_UNSUPPORTED;
+  if (N > (1 << 24)) return VS_ERR_UNSUPPORTED;
+  if (qs < (int64_t)Hq * d || kvs < (int64_t)Hkv * d) return VS_ERR_INVALID_ARG;
+  if (qs % 8 != 0 || kvs % 8 != 0) return VS_ERR_UNSUPPORTED;
+  if (!(scale >= 0.f) || std::isinf(scale)) return VS_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+    return VS_ERR_UNSUPPORTED;
+  return VS_OK;
+}
+
+}  // namespace vs
+
+using namespace vs;
+
+extern "C" {
+
+const char* vs_status_string(vs_status s) {
+  switch (s) {
+    case VS_OK: return "VS_OK";
+    case VS_ERR_INVALID_ARG: return "VS_ERR_INVALID_ARG";
+    case VS_ERR_UNSUPPORTED: return "VS_ERR_UNSUPPORTED";
+    case VS_ERR_WORKSPACE: return "VS_ERR_WORKSPACE";
+    case VS_ERR_CUDA: return "VS_ERR_CUDA";
+    case VS_ERR_DEVICE_TIMEOUT: return "VS_ERR_DEVICE_TIMEOUT";
+    case VS_ERR_DEVICE_BOUNDS: return "VS_ERR_DEVICE_BOUNDS";
+  }
+  return "VS_ERR_UNKNOWN";
+}
+
+int vs_version(void) { return 100; }
+
+vs_status vs_index_scores(const void* K, const void* V, vs_dtype dtype, int N, int Hkv, int d,
+                          int64_t stride_tok, int64_t stride_head, const float* W1,
+                          const float* W2, int hidden, float* logits_v, float* logits_s,
+                          cudaStream_t stream) {
+  if (!K || !V || !W1 || !W2 || !logits_v || !logits_s) return VS_ERR_INVALID_ARG;
+  if (dtype != VS_BF16 && dtype != VS_FP32) return VS_ERR_INVALID_ARG;
+  if (N < 1 || Hkv < 1 || d < 1 || d > 1024 || hidden < 1 || hidden > 1024)
+    return VS_ERR_INVALID_ARG;
+  if (stride_head < d || stride_tok < (int64_t)(Hkv - 1) * stride_head + d) return VS_ERR_INVALID_ARG;
+  if ((int64_t)N * Hkv > (int64_t)1 << 40) return VS_ERR_UNSUPPORTED;
+  if (launch_index_scores(K, V, dtype, N, Hkv, d, stride_tok, stride_head, W1, W2, hidden,
+                          logits_v, logits_s, stream) != cudaSuccess)
+    return VS_ERR_CUDA;
+  return VS_OK;
+}
+
+size_t vs_select_workspace_size(int H, int N) {
+  (void)H;
+  (void)N;
+  return kStatusBytes;
+}
+
+vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_select_mode mode,
+                    int k_or_cap, double tau, int32_t* idx, int64_t ld_idx, int32_t* count,
+                    void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!scores || !idx || !count) return VS_ERR_INVALID_ARG;
+  if (H < 1 || H > 65535 || N < 1 || ld_scores < N) return VS_ERR_INVALID_ARG;
+  if (N > (1 << 20)) return VS_ERR_UNSUPPORTED;
+  if (mode != VS_SELECT_TOPK && mode != VS_SELECT_THRESHOLD) return VS_ERR_INVALID_ARG;
+  if (k_or_cap < 1 || k_or_cap > N || ld_idx < k_or_cap) return VS_ERR_INVALID_ARG;
+  if (mode == VS_SELECT_THRESHOLD && !(tau > 0.0 && tau <= 1.0)) return VS_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < vs_select_workspace_size(H, N) || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  if (launch_select(scores, H, N, ld_scores, mode, k_or_cap, tau, idx, ld_idx, count, status,
+                    stream) != cudaSuccess)
+    return VS_ERR_CUDA;
+  return VS_OK;
+}
+
+size_t vs_attn_workspace_size(int N, int Hq, int H_sel, int d) {
+  (void)Hq;
+  (void)d;
+  if (N < 1 || H_sel < 1) return kStatusBytes;
+  return PlanLayout::make(N, H_sel).total;
+}
+
+static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
+                           int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                           float softmax_scale, bool sparse, int H_sel, const int32_t* v_idx,
+                           int64_t v_ld, const int32_t* v_cnt, const int32_t* s_idx, int64_t s_ld,
+                           const int32_t* s_cnt, void* O, float* lse, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+  vs_status st = check_attn_common(Q, K, V, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
+                                   softmax_scale, O);
+  if (st != VS_OK) return st;
+  if (sparse) {
+    if (!v_idx || !v_cnt || !s_idx || !s_cnt) return VS_ERR_INVALID_ARG;
+    if (N > (1 << 22)) return VS_ERR_UNSUPPORTED;  // plan kernel's block-diagonal bitmap
+    if (H_sel < 1 || Hq % H_sel != 0 || v_ld < 1 || s_ld < 1) return VS_ERR_INVALID_ARG;
+  } else {
+    H_sel = 1;
+  }
+  const size_t need = sparse ? vs_attn_workspace_size(N, Hq, H_sel, d) : kStatusBytes;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
+  AttnArgs a;
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.O = O;
+  a.lse = lse;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.H_sel = H_sel;
+  a.q_stride = q_stride_tok;
+  a.kv_stride = kv_stride_tok;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+  a.sparse = sparse;
+  a.v_idx = v_idx;
+  a.v_ld = v_ld;
+  a.v_cnt = v_cnt;
+  a.s_idx = s_idx;
+  a.s_ld = s_ld;
+  a.s_cnt = s_cnt;
+  a.ws = ws;
+  a.status = static_cast<int*>(ws);
+  a.stream = stream;
+  const PlanLayout L = PlanLayout::make(N, H_sel);
+  if (cudaMemsetAsync(a.status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  if (sparse && launch_plan(a, L) != cudaSuccess) return VS_ERR_CUDA;
+  cudaError_t e = dtype == VS_BF16 ? launch_attn_tc(a, L) : launch_attn_fp32(a, L);
+  return e == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
+vs_status vs_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
+                             int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                             float softmax_scale, int H_sel, const int32_t* v_idx, int64_t v_ld,
+                             const int32_t* v_cnt, const int32_t* s_idx, int64_t s_ld,
+                             const int32_t* s_cnt, void* O, float* lse, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+  return attn_impl(Q, K, V, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok, softmax_scale,
+                   true, H_sel, v_idx, v_ld, v_cnt, s_idx, s_ld, s_cnt, O, lse, ws, ws_bytes,
+                   stream);
+}
+
+vs_status vs_dense_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
+                            int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                            float softmax_scale, void* O, float* lse, void* ws, size_t ws_bytes,
+                            cudaStream_t stream) {
+  return attn_impl(Q, K, V, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok, softmax_scale,
+                   false, 1, nullptr, 0, nullptr, nullptr, 0, nullptr, O, lse, ws, ws_bytes,
+                   stream);
+}
+
+vs_status vs_read_device_status(const void* ws, cudaStream_t stream, int* flags) {
+  if (!ws || !flags) return VS_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return VS_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return VS_ERR_CUDA;
+  *flags = v;
+  if (v & VS_DEVFLAG_TIMEOUT) return VS_ERR_DEVICE_TIMEOUT;
+  if (v & VS_DEVFLAG_BOUNDS) return VS_ERR_DEVICE_BOUNDS;
+  return VS_OK;
+}
+
+vs_status vs_selftest_wait_timeout(void* ws, uint64_t limit_ns, cudaStream_t stream) {
+  if (!ws || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
+  if (limit_ns < 1000ull || limit_ns > 10000000000ull) return VS_ERR_INVALID_ARG;
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  return launch_wait_selftest(status, limit_ns, stream) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
+}  // extern "C"

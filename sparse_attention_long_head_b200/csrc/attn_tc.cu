@@ -1,0 +1,727 @@
+// Vertical-slash sparse (and dense causal) attention forward on sm_100a.
+//
+// What is computed follows the VSPrefill summary pages, "VSPrefill ..."
+// Technical Summary, section 2: each query attends to the union of the
+// selected vertical key columns and the keys at the selected slash offsets
+// behind it, inside one FlashAttention-style kernel with no precomputed mask.
+// How it is computed is this library's own design for B200:
+//
+//   * A plan kernel turns the index lists into per-head bitmaps (columns,
+//     offsets), an ascending column list, and the list of touched
+//     block-diagonals.  No n x n structure is ever built.
+//   * The attention kernel is persistent: one CTA per SM walks "units" of 256
+//     query rows of one head (two 128-row sub-tiles A and B), heaviest first.
+//   * Per unit it streams "items": 128-key blocks loaded by TMA (tiled), or
+//     128-column chunks of the vertical list gathered row by row with TMA
+//     tile::gather4.  Each item is applied to both sub-tiles.
+//   * QK^T and PV run on tcgen05 (bf16 in, fp32 accumulate in TMEM); P is
+//     written back into TMEM over S and consumed by the TS-form MMA.
+//   * Four softmax warps per sub-tile own one row each; the element mask of a
+//     key block is four 32-bit words per row read from the offset and column
+//     bitmaps, so a key that is both a column and on a selected diagonal is
+//     counted once.  Online softmax with lazy rescaling of O (only when the
+//     running max grows by more than 2^8).
+//   * Per unit the plan picks, in O(1), the cheaper of: every key block of
+//     the causal triangle with mask (S or V) ("dense-vs"), or the gathered
+//     vertical chunks plus only the key blocks on touched block-diagonals with
+//     mask (S and not V) ("split").
+//
+// Warp roles (320 threads): warps 0-3 softmax/epilogue of sub-tile A, warps
+// 4-7 of sub-tile B, warp 8 issues the MMAs (one thread) and owns TMEM,
+// warp 9 issues the TMA loads.  Every wait is bounded (see WaitCtx).
+#include <cstdio>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vs {
+
+// ------------------------------------------------------------------ plan
+
+// Writes, in ascending order, the positions of the set bits of
+// bits[0 .. nwords) (bit positions < limit) to out[]; returns the count.
+// Whole block participates; `scan` is blockDim.x ints of shared memory.
+__device__ int block_bits_to_list(const uint32_t* bits, int64_t nwords, int64_t limit,
+                                  int32_t* out, int* scan) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int64_t per = (nwords + nt - 1) / nt;
+  const int64_t w0 = tid * per, w1 = min(nwords, w0 + per);
+  int c = 0;
+  for (int64_t w = w0; w < w1; ++w) c += __popc(bits[w]);
+  scan[tid] = c;
+  __syncthreads();
+  for (int off = 1; off < nt; off <<= 1) {
+    int v = tid >= off ? scan[tid - off] : 0;
+    __syncthreads();
+    scan[tid] += v;
+    __syncthreads();
+  }
+  int pos = scan[tid] - c;
+  const int total = scan[nt - 1];
+  for (int64_t w = w0; w < w1; ++w) {
+    uint32_t x = bits[w];
+    while (x) {
+      int b = __ffs(x) - 1;
+      x &= x - 1;
+      int64_t v = w * 32 + b;
+      if (v < limit) out[pos] = static_cast<int32_t>(v);
+      ++pos;
+    }
+  }
+  __syncthreads();
+  return total;
+}
+
+struct PlanKernelArgs {
+  int N, H_sel;
+  const int32_t* v_idx;
+  int64_t v_ld;
+  const int32_t* v_cnt;
+  const int32_t* s_idx;
+  int64_t s_ld;
+  const int32_t* s_cnt;
+  void* ws;
+  int* status;
+  PlanLayout L;
+};
+
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanKernelArgs a) {
+  __shared__ int scan[kPlanThreads];
+  __shared__ uint32_t dbits[1026];  // touched block-diagonals, T <= 32768
+  __shared__ uint32_t d1bits[1026];
+  __shared__ int bad;
+  const int hs = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+  const PlanLayout& L = a.L;
+  PlanPtrs pp = plan_ptrs(L, a.ws);
+  uint32_t* vb = pp.vbits + (int64_t)hs * L.vbits_words;
+  uint32_t* sb = pp.sbits + (int64_t)hs * L.sbits_words;
+  const int N = a.N, T = L.T;
+  const int dwords = (T + 2 + 31) / 32;
+  for (int64_t w = tid; w < L.vbits_words; w += nt) vb[w] = 0;
+  for (int64_t w = tid; w < L.sbits_words; w += nt) sb[w] = 0;
+  for (int w = tid; w < dwords; w += nt) dbits[w] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+
+  int nv_in = a.v_cnt[hs], ns_in = a.s_cnt[hs];
+  if (nv_in < 0 || nv_in > a.v_ld) {
+    nv_in = nv_in < 0 ? 0 : (int)a.v_ld;
+    bad = 1;
+  }
+  if (ns_in < 0 || ns_in > a.s_ld) {
+    ns_in = ns_in < 0 ? 0 : (int)a.s_ld;
+    bad = 1;
+  }
+  for (int t = tid; t < nv_in; t += nt) {
+    int j = a.v_idx[(int64_t)hs * a.v_ld + t];
+    if (j >= 0 && j < N) atomicOr(&vb[j >> 5], 1u << (j & 31));
+    else bad = 1;
+  }
+  for (int t = tid; t < ns_in; t += nt) {
+    int o = a.s_idx[(int64_t)hs * a.s_ld + t];
+    if (o >= 0 && o < N) {
+      int pos = N - o + 128;
+      atomicOr(&sb[pos >> 5], 1u << (pos & 31));
+      int dl = o >> 7;
+      atomicOr(&dbits[dl >> 5], 1u << (dl & 31));
+      if ((o & 127) && dl + 1 < T) atomicOr(&dbits[(dl + 1) >> 5], 1u << ((dl + 1) & 31));
+    } else {
+      bad = 1;
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && bad) atomicOr(a.status, VS_DEVFLAG_BOUNDS);
+  // d' in [0, T] is needed iff d' or d'-1 is touched.
+  for (int w = tid; w < dwords; w += nt) {
+    uint32_t cur = dbits[w], prev = w > 0 ? dbits[w - 1] : 0u;
+    d1bits[w] = cur | (cur << 1) | (prev >> 31);
+  }
+  __syncthreads();
+  int32_t* vlist = pp.vlist + (int64_t)hs * N;
+  int32_t* slist = pp.slist + (int64_t)hs * N;
+  int32_t* d1list = pp.d1list + (int64_t)hs * L.d1_len;
+  int32_t* d1pref = pp.d1pref + (int64_t)hs * L.d1pref_len;
+  int32_t* vpair = pp.vpair + (int64_t)hs * L.vpair_len;
+  const int nv = block_bits_to_list(vb, (N + 31) / 32, N, vlist, scan);
+  // offsets ascending = positions N - o + 128 descending: collect, then reverse.
+  int ns = 0;
+  {
+    // positions live in [129, N + 128]; list them ascending into slist, then
+    // map pos -> o = N + 128 - pos and reverse in place.
+    ns = block_bits_to_list(sb, L.sbits_words, (int64_t)N + 129, slist, scan);
+    for (int t = tid; t < ns / 2; t += nt) {
+      int x = slist[t], y = slist[ns - 1 - t];
+      slist[t] = N + 128 - y;
+      slist[ns - 1 - t] = N + 128 - x;
+    }
+    if ((ns & 1) && tid == 0) slist[ns / 2] = N + 128 - slist[ns / 2];
+    __syncthreads();
+  }
+  {
+    const int nd1 = block_bits_to_list(d1bits, (T + 1 + 31) / 32, (int64_t)T + 1, d1list, scan);
+    for (int x = tid; x < L.d1pref_len; x += nt) {
+      int lo = 0, hi = nd1;  // lower_bound(d1list, x)
+      while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (d1list[mid] < x) lo = mid + 1;
+        else hi = mid;
+      }
+      d1pref[x] = lo;
+    }
+    for (int p = tid; p < L.P; p += nt) {
+      int lim = min(256 * p + 255, N - 1);
+      int lo = 0, hi = nv;  // upper_bound(vlist, lim)
+      while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (vlist[mid] <= lim) lo = mid + 1;
+        else hi = mid;
+      }
+      vpair[p] = lo;
+    }
+    if (tid == 0) {
+      int32_t* m = pp.meta + 4 * hs;
+      m[0] = nv;
+      m[1] = ns;
+      m[2] = nd1;
+      m[3] = 0;
+    }
+  }
+}
+
+cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L) {
+  if (L.T + 2 > 1026 * 32) return cudaErrorInvalidValue;
+  PlanKernelArgs k{a.N, a.H_sel, a.v_idx, a.v_ld, a.v_cnt, a.s_idx, a.s_ld, a.s_cnt, a.ws, a.status, L};
+  plan_kernel<<<a.H_sel, kPlanThreads, 0, a.stream>>>(k);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------- attention
+
+constexpr int kAttnThreads = 320;
+constexpr int kWarpMMA = 8;
+constexpr int kWarpLoad = 9;
+
+enum : int { kModeDense = 0, kModeDenseVS = 1, kModeSplit = 2 };
+enum : int { kItemTile = 0, kItemVChunk = 1 };
+
+template <int D>
+struct Cfg {
+  static constexpr int kTileBytes = 128 * D * 2;  // one 128-row K or V tile
+  static constexpr int kStages = D == 128 ? 4 : 8;
+  static constexpr int kQBytes = kTileBytes;
+  static constexpr int kData = 2 * kQBytes + kStages * kTileBytes;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmem = kData + kBarBytes + 1024;  // + alignment slack
+};
+
+struct AttnParams {
+  int N, Hq, Hkv, H_sel, T, P, G;
+  int num_units;
+  int64_t q_stride;
+  float scale_log2;  // softmax scale * log2(e)
+  __nv_bfloat16* O;
+  float* lse;
+  int* status;
+  uint64_t wait_limit_ns;
+  PlanLayout L;
+  PlanPtrs pp;
+};
+
+struct UnitInfo {
+  int h, hs, g, p, n, mode, nvc, nv, d1start;
+};
+
+template <bool SPARSE>
+__device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
+  UnitInfo ui;
+  ui.p = P.P - 1 - u / P.Hq;
+  ui.h = u % P.Hq;
+  ui.g = ui.h / P.G;
+  ui.hs = (int)(((int64_t)ui.h * P.H_sel) / P.Hq);
+  const int last_b = min(2 * ui.p + 1, P.T - 1);
+  const int n_dense = last_b + 1;
+  ui.nvc = 0;
+  ui.nv = 0;
+  ui.d1start = 0;
+  if (!SPARSE) {
+    ui.mode = kModeDense;
+    ui.n = n_dense;
+    return ui;
+  }
+  const int32_t* d1pref = P.pp.d1pref + (int64_t)ui.hs * P.L.d1pref_len;
+  // key block b = 2p+1-d' must lie in [0, last_b]  =>  d' in [2p+1-last_b, 2p+1]
+  const int lo = 2 * ui.p + 1 - last_b, hi = 2 * ui.p + 1;
+  const int nslash = d1pref[hi + 1] - d1pref[lo];
+  const int nvp = P.pp.vpair[(int64_t)ui.hs * P.L.vpair_len + ui.p];
+  const int nvc = (nvp + 127) / 128;
+  if (nvc + nslash < n_dense) {
+    ui.mode = kModeSplit;
+    ui.n = nvc + nslash;
+    ui.nvc = nvc;
+    ui.nv = P.pp.meta[4 * ui.hs + 0];
+    ui.d1start = d1pref[lo];
+  } else {
+    ui.mode = kModeDenseVS;
+    ui.n = n_dense;
+  }
+  return ui;
+}
+
+struct Item {
+  int kind;
+  int b;  // key block (tile) or chunk index (vertical chunk)
+};
+
+__device__ __forceinline__ Item unit_item(const AttnParams& P, const UnitInfo& ui, int k) {
+  Item it;
+  if (ui.mode != kModeSplit) {
+    it.kind = kItemTile;
+    it.b = k;
+  } else if (k < ui.nvc) {
+    it.kind = kItemVChunk;
+    it.b = k;
+  } else {
+    it.kind = kItemTile;
+    it.b = 2 * ui.p + 1 - P.pp.d1list[(int64_t)ui.hs * P.L.d1_len + ui.d1start + (k - ui.nvc)];
+  }
+  return it;
+}
+
+__device__ __forceinline__ uint32_t prefix_word(int n, int lo) {
+  // bits [0, n - lo) of the 32-bit word covering positions [lo, lo + 32)
+  const int k = n - lo;
+  return k <= 0 ? 0u : (k >= 32 ? 0xffffffffu : ((1u << k) - 1u));
+}
+
+// 128-bit keep-mask of row i for one item; returns false if every key is kept.
+template <bool SPARSE>
+__device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& ui, const Item& it,
+                                          int i, int t_sub, uint32_t (&w)[4]) {
+  if (it.kind == kItemVChunk) {
+    const int32_t* base = P.pp.vlist + (int64_t)ui.hs * P.N + 128 * it.b;
+    const int cnt = min(128, ui.nv - 128 * it.b);
+    int n = cnt;
+    if (base[cnt - 1] > i) {
+      int lo = 0, hi = cnt;
+      while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (base[mid] <= i) lo = mid + 1;
+        else hi = mid;
+      }
+      n = lo;
+    }
+    if (n == 128) return false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = prefix_word(n, 32 * q);
+    return true;
+  }
+  const int b = it.b;
+  // causal part for the keys of block b: keep c <= i - 128 b
+  const bool below = b < t_sub;  // whole block in the past of every row of the sub-tile
+  if (!SPARSE || ui.mode == kModeDense) {
+    if (below) return false;
+    const int n = i - 128 * b + 1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = prefix_word(n, 32 * q);
+    return true;
+  }
+  // offset window: bit c = [ i - (128 b + c) is a selected offset ]
+  const uint32_t* sb = P.pp.sbits + (int64_t)ui.hs * P.L.sbits_words;
+  const int64_t pos0 = (int64_t)P.N - i + 128 + 128 * b;
+  const uint32_t* sw = sb + (pos0 >> 5);
+  const int sh = (int)(pos0 & 31);
+  uint32_t x[5];
+#pragma unroll
+  for (int q = 0; q < 5; ++q) x[q] = __ldg(sw + q);
+  uint32_t s[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) s[q] = __funnelshift_r(x[q], x[q + 1], sh);
+  const uint32_t* vb = P.pp.vbits + (int64_t)ui.hs * P.L.vbits_words + 4 * b;
+  if (ui.mode == kModeDenseVS) {
+    const int n = below ? 128 : i - 128 * b + 1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = s[q] | (__ldg(vb + q) & prefix_word(n, 32 * q));
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = s[q] & ~__ldg(vb + q);
+  }
+  return true;
+}
+
+template <int D, bool SPARSE>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKg,
+                   const __grid_constant__ CUtensorMap tmVg, const AttnParams P) {
+  using C = Cfg<D>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + 2 * C::kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kData);
+  enum { B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 6, B_OEMPTY = 8,
+         B_DRAIN = 10, B_FULL = 11, B_EMPTY = 11 + S, B_END = 11 + 2 * S };
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + B_END);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QEMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_SFULL + s), 1);
+      mbar_init(bar(B_PFULL + s), 128);
+      mbar_init(bar(B_OFULL + s), 1);
+      mbar_init(bar(B_OEMPTY + s), 128);
+    }
+    mbar_init(bar(B_DRAIN), 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    if (SPARSE) {
+      tma_prefetch_desc(&tmKg);
+      tma_prefetch_desc(&tmVg);
+    }
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(smem_u32(tslot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  const WaitCtx wc{P.wait_limit_ns, P.status, abort_flag};
+
+  if (warp < 8) {
+    // ------------------------------------------------ softmax + epilogue
+    const int sub = warp >> 2;
+    const int r = tid & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tbase + lane_off + sub * 128;
+    const uint32_t tO = tbase + lane_off + 256 + sub * 128;
+    uint32_t scnt = 0, ucount = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
+      const UnitInfo ui = unit_info<SPARSE>(P, u);
+      const int i = 256 * ui.p + 128 * sub + r;
+      const int im = min(i, P.N - 1);
+      const int t_sub = 2 * ui.p + sub;
+      __nv_bfloat16* orow = P.O + (int64_t)i * P.q_stride + (int64_t)ui.h * D;
+      if (ui.n == 0) {
+        if (i < P.N) {
+          for (int c = 0; c < D; c += 8)
+            *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+          if (P.lse) P.lse[(int64_t)ui.h * P.N + i] = -INFINITY;
+        }
+        continue;
+      }
+      float m_use = -INFINITY, l = 0.f;
+      for (int k = 0; k < ui.n; ++k) {
+        const Item it = unit_item(P, ui, k);
+        uint32_t mw[4];
+        const bool masked = item_mask<SPARSE>(P, ui, it, im, t_sub, mw);
+        if (!mbar_wait(bar(B_SFULL + sub), scnt & 1, wc)) { ok = false; break; }
+        ++scnt;
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, sr[q]);
+        tmem_ld_wait(sr[0]);
+        reg_pin(sr[1]);
+        reg_pin(sr[2]);
+        reg_pin(sr[3]);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            float v = __uint_as_float(sr[q][c]);
+            if (masked && !((mw[q] >> c) & 1u)) v = -INFINITY;
+            sr[q][c] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        }
+        const float m_cand = mx * P.scale_log2;
+        const bool need = m_cand > m_use + 8.0f;
+        float factor = 1.f;
+        if (need) {
+          factor = ex2_approx(m_use - m_cand);  // 0 when m_use = -inf
+          m_use = m_cand;
+          l *= factor;
+        }
+        const float m_base = m_use == -INFINITY ? 0.f : m_use;
+        float ls = 0.f;
+        uint32_t pk[2][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][c]), P.scale_log2, -m_base));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][c + 1]), P.scale_log2, -m_base));
+            ls += p0 + p1;
+            pk[q >> 1][(q & 1) * 16 + c / 2] = pack_bf16x2(p0, p1);
+          }
+        }
+        l += ls;
+        tmem_st32(tS, pk[0]);
+        tmem_st32(tS + 32, pk[1]);
+        if (k > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * q, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+            tmem_st32(tO + 32 * q, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + sub));
+      }
+      if (!ok) break;
+      if (!mbar_wait(bar(B_OFULL + sub), ucount & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * q, o);
+        tmem_ld_wait(o);
+        if (i < P.N) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + 32 * q + c) = v;
+          }
+        }
+      }
+      if (i < P.N && P.lse)
+        P.lse[(int64_t)ui.h * P.N + i] =
+            l > 0.f ? (m_use + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      tc_fence_before();
+      mbar_arrive(bar(B_OEMPTY + sub));
+      ++ucount;
+    }
+  } else if (warp == kWarpMMA) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+      const uint32_t q_addr = smem_u32(sQ), kv_addr = smem_u32(sKV);
+      uint32_t seq = 0, ucount = 0, pcnt[2] = {0, 0};
+      bool ok = true;
+      auto issue_s = [&](int sub, uint32_t slot) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint64_t ad = sdesc_sw128(q_addr + sub * C::kQBytes + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kv_addr + slot * C::kTileBytes + off, 16, 1024);
+          mma_ss(tbase + sub * 128, ad, bd, idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int sub, uint32_t slot, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = sdesc_sw128(kv_addr + slot * C::kTileBytes + kk * 2048, 16384, 1024);
+          mma_ts(tbase + 256 + sub * 128, tbase + sub * 128 + kk * 8, bd, idesc_pv,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
+        const UnitInfo ui = unit_info<SPARSE>(P, u);
+        if (ui.n == 0) continue;
+        if (!mbar_wait(bar(B_QFULL), ucount & 1, wc)) { ok = false; break; }
+        uint32_t kslot = seq % S;
+        if (!mbar_wait(bar(B_FULL + kslot), (seq / S) & 1, wc)) { ok = false; break; }
+        ++seq;
+        tc_fence_after();
+        issue_s(0, kslot);
+        mma_commit(bar(B_SFULL + 0));
+        issue_s(1, kslot);
+        mma_commit(bar(B_SFULL + 1));
+        mma_commit(bar(B_EMPTY + kslot));
+        for (int k = 0; k < ui.n && ok; ++k) {
+          const uint32_t vslot = seq % S;
+          if (!mbar_wait(bar(B_FULL + vslot), (seq / S) & 1, wc)) { ok = false; break; }
+          ++seq;
+          for (int sub = 0; sub < 2; ++sub) {
+            if (!mbar_wait(bar(B_PFULL + sub), pcnt[sub] & 1, wc)) { ok = false; break; }
+            ++pcnt[sub];
+            if (k == 0 && ucount > 0) {
+              if (!mbar_wait(bar(B_OEMPTY + sub), (ucount - 1) & 1, wc)) { ok = false; break; }
+            }
+            tc_fence_after();
+            issue_pv(sub, vslot, k > 0);
+            if (sub == 1) mma_commit(bar(B_EMPTY + vslot));
+            if (k + 1 < ui.n) {
+              if (sub == 0) {
+                kslot = seq % S;
+                if (!mbar_wait(bar(B_FULL + kslot), (seq / S) & 1, wc)) { ok = false; break; }
+                ++seq;
+                tc_fence_after();
+              }
+              issue_s(sub, kslot);
+              mma_commit(bar(B_SFULL + sub));
+              if (sub == 1) mma_commit(bar(B_EMPTY + kslot));
+            } else {
+              mma_commit(bar(B_OFULL + sub));
+            }
+          }
+        }
+        if (!ok) break;
+        mma_commit(bar(B_QEMPTY));
+        ++ucount;
+      }
+      // Drain: every MMA issued so far must finish before TMEM is freed.
+      mma_commit(bar(B_DRAIN));
+      mbar_wait_drain(bar(B_DRAIN), 0, P.wait_limit_ns);
+    }
+  } else if (warp == kWarpLoad) {
+    // ------------------------------------------------------- TMA producer
+    uint32_t seq = 0, ucount = 0;
+    bool ok = true;
+    const int nsub64 = D / 64;
+    for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
+      const UnitInfo ui = unit_info<SPARSE>(P, u);
+      if (ui.n == 0) continue;
+      if (ucount > 0 && !mbar_wait(bar(B_QEMPTY), (ucount - 1) & 1, wc)) { ok = false; break; }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kQBytes);
+        for (int s = 0; s < 2; ++s)
+          for (int h = 0; h < nsub64; ++h)
+            tma_load_2d(smem_u32(sQ + s * C::kQBytes + h * 16384), &tmQ, bar(B_QFULL),
+                        ui.h * D + 64 * h, 256 * ui.p + 128 * s);
+      }
+      ++ucount;
+      for (int k = 0; k < ui.n && ok; ++k) {
+        const Item it = unit_item(P, ui, k);
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t slot = seq % S;
+          if (seq >= (uint32_t)S && !mbar_wait(bar(B_EMPTY + slot), ((seq / S) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar(B_FULL + slot);
+          if (lane == 0) mbar_arrive_expect_tx(fb, C::kTileBytes);
+          __syncwarp();
+          const uint32_t dst = smem_u32(sKV + slot * C::kTileBytes);
+          if (it.kind == kItemTile) {
+            if (lane == 0) {
+              const CUtensorMap* m = kv ? &tmV : &tmK;
+              for (int h = 0; h < nsub64; ++h)
+                tma_load_2d(dst + h * 16384, m, fb, ui.g * D + 64 * h, 128 * it.b);
+            }
+          } else {
+            const int32_t* base = P.pp.vlist + (int64_t)ui.hs * P.N + 128 * it.b;
+            const int cnt = min(128, ui.nv - 128 * it.b);
+            int rr[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int e = 4 * lane + q;
+              rr[q] = base[e < cnt ? e : 0];
+            }
+            const CUtensorMap* m = kv ? &tmVg : &tmKg;
+            for (int h = 0; h < nsub64; ++h)
+              tma_gather4(dst + h * 16384 + lane * 512, m, fb, ui.g * D + 64 * h, rr[0], rr[1],
+                          rr[2], rr[3]);
+          }
+          ++seq;
+        }
+      }
+    }
+    // Drain: let every issued copy land before shared memory is released.
+    if (lane == 0) {
+      const uint32_t first = seq > (uint32_t)S ? seq - S : 0;
+      for (uint32_t x = first; x < seq; ++x)
+        mbar_wait_drain(bar(B_FULL + (x % S)), (x / S) & 1, P.wait_limit_ns);
+      if (ucount > 0) mbar_wait_drain(bar(B_QFULL), (ucount - 1) & 1, P.wait_limit_ns);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+
+static void encode_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t inner,
+                       int64_t rows, int64_t row_stride_elems, uint32_t box_rows, CUresult* rc) {
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) *rc = r;
+}
+
+template <int D, bool SPARSE>
+static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap mQ, mK, mV, mKg, mVg;
+  CUresult rc = CUDA_SUCCESS;
+  encode_map(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.N, a.q_stride, 128, &rc);
+  encode_map(enc, &mK, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, 128, &rc);
+  encode_map(enc, &mV, a.V, (int64_t)a.Hkv * D, a.N, a.kv_stride, 128, &rc);
+  encode_map(enc, &mKg, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
+  encode_map(enc, &mVg, a.V, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
+  if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  AttnParams P;
+  P.N = a.N;
+  P.Hq = a.Hq;
+  P.Hkv = a.Hkv;
+  P.H_sel = SPARSE ? a.H_sel : 1;
+  P.T = L.T;
+  P.P = L.P;
+  P.G = a.Hq / a.Hkv;
+  P.num_units = a.Hq * L.P;
+  P.q_stride = a.q_stride;
+  P.scale_log2 = a.scale * 1.4426950408889634f;
+  P.O = static_cast<__nv_bfloat16*>(a.O);
+  P.lse = a.lse;
+  P.status = a.status;
+  P.wait_limit_ns = kDefaultWaitLimitNs;
+  P.L = L;
+  P.pp = plan_ptrs(L, a.ws);
+  auto kern = attn_tc_kernel<D, SPARSE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<D>::kSmem);
+  if (e != cudaSuccess) return e;
+  const int grid = P.num_units < device_sm_count() ? P.num_units : device_sm_count();
+  kern<<<grid, kAttnThreads, Cfg<D>::kSmem, a.stream>>>(mQ, mK, mV, mKg, mVg, P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, const PlanLayout& L) {
+  if (a.d == 128) return a.sparse ? launch_tc_impl<128, true>(a, L) : launch_tc_impl<128, false>(a, L);
+  if (a.d == 64) return a.sparse ? launch_tc_impl<64, true>(a, L) : launch_tc_impl<64, false>(a, L);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vs

@@ -1,0 +1,142 @@
+// Internal declarations shared by the host API and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "vs_prefill.h"
+
+namespace vs {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+constexpr size_t kStatusBytes = 256;                      // status word + padding
+
+inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Per-index-set-head plan data written by the plan kernel into the
+// workspace (after the status header).  All sizes depend on N only.
+//   vbits  : column bitmap, bit j set iff j is a selected column, padded with
+//            zero bits up to 128*T + 128.
+//   sbits  : offset bitmap in "reversed" positions: bit (N - o + 128) set iff
+//            o is a selected offset; zero elsewhere.  A 128-bit window read at
+//            position N - i + 128 + 128*b gives, for row i and key block b,
+//            bit c = [ (i - (128b + c)) is a selected offset ], which is 0 for
+//            every key in the future of i.
+//   vlist  : selected columns ascending, deduplicated (N entries reserved).
+//   slist  : selected offsets ascending, deduplicated (N entries reserved).
+//   d1list : ascending list of block-diagonal indices d' in [0, T] such that
+//            d' or d'-1 is "touched" (a selected offset lies in
+//            [128 d - 127, 128 d + 127]).  A 256-row unit at pair p needs key
+//            block b iff 2p+1-b is in this list.
+//   d1pref : d1pref[x] = #{ d' in d1list : d' < x }, x in [0, T+1].
+//   vpair  : vpair[p] = #{ j in vlist : j <= min(256 p + 255, N - 1) }.
+//   meta   : [nv, ns, nd1, 0].
+struct PlanLayout {
+  int N = 0, T = 0, P = 0, H = 0;
+  int64_t vbits_words = 0, sbits_words = 0, d1_len = 0, d1pref_len = 0, vpair_len = 0;
+  size_t off_meta = 0, off_vbits = 0, off_sbits = 0, off_vlist = 0, off_slist = 0,
+         off_d1list = 0, off_d1pref = 0, off_vpair = 0, total = 0;
+
+  __host__ __device__ static PlanLayout make(int N, int H) {
+    PlanLayout L;
+    L.N = N;
+    L.H = H;
+    L.T = (N + 127) / 128;
+    L.P = (L.T + 1) / 2;
+    L.vbits_words = 4 * (int64_t)(L.T + 2);
+    L.sbits_words = ((int64_t)N + 512 + 31) / 32 + 2;
+    L.d1_len = L.T + 1;
+    L.d1pref_len = L.T + 2;
+    L.vpair_len = L.P;
+    size_t off = 256;  // status header
+    auto take = [&](size_t bytes) {
+      size_t o = off;
+      off = (off + bytes + 255) / 256 * 256;
+      return o;
+    };
+    L.off_meta = take(sizeof(int32_t) * 4 * (size_t)H);
+    L.off_vbits = take(sizeof(uint32_t) * (size_t)L.vbits_words * H);
+    L.off_sbits = take(sizeof(uint32_t) * (size_t)L.sbits_words * H);
+    L.off_vlist = take(sizeof(int32_t) * (size_t)N * H);
+    L.off_slist = take(sizeof(int32_t) * (size_t)N * H);
+    L.off_d1list = take(sizeof(int32_t) * (size_t)L.d1_len * H);
+    L.off_d1pref = take(sizeof(int32_t) * (size_t)L.d1pref_len * H);
+    L.off_vpair = take(sizeof(int32_t) * (size_t)L.vpair_len * H);
+    L.total = off;
+    return L;
+  }
+};
+
+struct PlanPtrs {
+  int32_t* meta;
+  uint32_t* vbits;
+  uint32_t* sbits;
+  int32_t* vlist;
+  int32_t* slist;
+  int32_t* d1list;
+  int32_t* d1pref;
+  int32_t* vpair;
+};
+
+inline __host__ __device__ PlanPtrs plan_ptrs(const PlanLayout& L, void* ws) {
+  char* b = static_cast<char*>(ws);
+  PlanPtrs p;
+  p.meta = reinterpret_cast<int32_t*>(b + L.off_meta);
+  p.vbits = reinterpret_cast<uint32_t*>(b + L.off_vbits);
+  p.sbits = reinterpret_cast<uint32_t*>(b + L.off_sbits);
+  p.vlist = reinterpret_cast<int32_t*>(b + L.off_vlist);
+  p.slist = reinterpret_cast<int32_t*>(b + L.off_slist);
+  p.d1list = reinterpret_cast<int32_t*>(b + L.off_d1list);
+  p.d1pref = reinterpret_cast<int32_t*>(b + L.off_d1pref);
+  p.vpair = reinterpret_cast<int32_t*>(b + L.off_vpair);
+  return p;
+}
+
+// Common attention launch description.
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  void* O;
+  float* lse;
+  int N, Hq, Hkv, d, H_sel;
+  int64_t q_stride, kv_stride;
+  float scale;
+  bool sparse;
+  const int32_t* v_idx;
+  int64_t v_ld;
+  const int32_t* v_cnt;
+  const int32_t* s_idx;
+  int64_t s_ld;
+  const int32_t* s_cnt;
+  void* ws;
+  int* status;
+  cudaStream_t stream;
+};
+
+// Launchers (return a CUDA error; argument checks are done by the caller).
+cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L);
+cudaError_t launch_attn_tc(const AttnArgs& a, const PlanLayout& L);
+cudaError_t launch_attn_fp32(const AttnArgs& a, const PlanLayout& L);
+cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,
+                          double tau, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
+                          cudaStream_t stream);
+cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, int Hkv, int d,
+                                int64_t stride_tok, int64_t stride_head, const float* W1,
+                                const float* W2, int hidden, float* lv, float* ls,
+                                cudaStream_t stream);
+cudaError_t launch_wait_selftest(int* status, uint64_t limit_ns, cudaStream_t stream);
+
+// Driver entry point for tensor-map encoding (resolved once through the
+// runtime; no link-time dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+int device_sm_count();
+
+}  // namespace vs

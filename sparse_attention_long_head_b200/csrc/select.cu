@@ -1,0 +1,336 @@
+// Per-head vertical / slash budget selection (top-k or cumulative mass) on
+// sm_100a.
+//
+// The rule is the VSPrefill pages' budget step ("VSPrefill ..." Technical
+// Summary, section 2, Adaptive Inference Pipeline, Dynamic Budgeting: a
+// cumulative threshold over the predicted scores decides how many indices to
+// keep; the German page's Inferenz-Pipeline phrases it as the number of top-k
+// indices needed to keep a given mass).  FlashPrefill's summary page
+// (section 1) notes that sorting and cumulative sums are what make such
+// selection expensive on GPUs; this kernel therefore never sorts:
+//
+//   * One thread-block cluster per head (C <= 8 CTAs); each CTA keeps its
+//     slice of the scores as order-preserving 32-bit keys in shared memory.
+//   * A most-significant-digit radix search (4 passes of 8 bits) finds the
+//     exact boundary key.  Per pass every CTA builds a 256-bucket histogram of
+//     counts (and, for the threshold rule, of fp64 softmax mass); the cluster
+//     merges them through distributed shared memory, and every CTA takes the
+//     same decision from the same merged data.
+//   * The threshold rule walks the buckets from the top, accumulating mass
+//     until tau * Z is reached; inside the final group of equal keys the
+//     count follows from their common mass.
+//   * A last pass writes the kept indices in ascending order (index-ordered
+//     compaction across the cluster), then pads with -1.
+#include <cooperative_groups.h>
+
+#include "internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace vs {
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelMaxCluster = 8;
+constexpr int kSelCacheKeys = 32768;  // 128 KB of keys per CTA
+
+// Order-preserving key: larger key = earlier in (score desc); NaN -> 0
+// (after everything, including -inf); -0.0 is folded onto +0.0.
+__device__ __forceinline__ uint32_t fkey(float f) {
+  if (f != f) return 0u;
+  if (f == 0.f) f = 0.f;
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float fkey_inv(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+struct SelArgs {
+  const float* scores;
+  int N;
+  int64_t ld;
+  int mode;
+  int k_or_cap;
+  double tau;
+  int32_t* idx;
+  int64_t ld_idx;
+  int32_t* count;
+  int* status;
+  int chunk;
+};
+
+struct SelShared {
+  uint32_t cnt[2][256];
+  double mass[2][256];
+  uint32_t tot_c[256];
+  double tot_m[256];
+  uint32_t kmax;
+  double zpart;
+  uint32_t npos;
+  uint32_t gt, eq;
+  int bstar;
+  uint32_t cabove, eqcnt;
+  double mabove;
+  int wred_i[32];
+  double wred_d[32];
+  int scan_a[kSelThreads];
+  int scan_b[kSelThreads];
+};
+
+__device__ __forceinline__ double pmass(uint32_t key, uint32_t kmax, double smax) {
+  if (key == kmax) return 1.0;
+  if (key == 0u) return 0.0;
+  return exp(static_cast<double>(fkey_inv(key)) - smax);
+}
+
+template <typename T, typename Op>
+__device__ __forceinline__ T block_reduce(T v, T* wred, Op op) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) wred[warp] = v;
+  __syncthreads();
+  T r = wred[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = op(r, wred[w]);
+  __syncthreads();
+  return r;
+}
+
+// Exclusive prefix sum over the block (int), returns this thread's prefix.
+__device__ __forceinline__ int block_excl_scan(int v, int* buf) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  buf[tid] = v;
+  __syncthreads();
+  for (int off = 1; off < nt; off <<= 1) {
+    int x = tid >= off ? buf[tid - off] : 0;
+    __syncthreads();
+    buf[tid] += x;
+    __syncthreads();
+  }
+  int r = buf[tid] - v;
+  __syncthreads();
+  return r;
+}
+
+template <bool CACHE>
+__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  const int C = static_cast<int>(cl.num_blocks());
+  const int h = blockIdx.y;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  extern __shared__ uint32_t skeys[];
+  __shared__ SelShared sh;
+
+  const float* row = a.scores + (int64_t)h * a.ld;
+  const int lo = rank * a.chunk;
+  const int n = max(0, min(a.N, lo + a.chunk) - lo);
+  auto key_at = [&](int e) -> uint32_t { return CACHE ? skeys[e] : fkey(__ldg(row + lo + e)); };
+
+  // ---- keys and the cluster-wide maximum key
+  uint32_t lmax = 0;
+  for (int e = tid; e < n; e += nt) {
+    const uint32_t k = fkey(__ldg(row + lo + e));
+    if (CACHE) skeys[e] = k;
+    lmax = max(lmax, k);
+  }
+  lmax = block_reduce<int>(static_cast<int>(lmax ^ 0x80000000u), sh.wred_i,
+                           [](int x, int y) { return x > y ? x : y; }) ^ 0x80000000u;
+  if (tid == 0) sh.kmax = lmax;
+  cl.sync();
+  uint32_t kmax = 0;
+  for (int r = 0; r < C; ++r) kmax = max(kmax, *cl.map_shared_rank(&sh.kmax, r));
+  const double smax = static_cast<double>(fkey_inv(kmax));
+
+  int mode = a.mode;
+  int k_target = a.k_or_cap;
+  double target = 0.0;
+  if (mode == VS_SELECT_THRESHOLD) {
+    if (kmax == 0u) {  // every score is NaN: keep one entry
+      mode = VS_SELECT_TOPK;
+      k_target = 1;
+    } else if (a.tau >= 1.0) {  // keep every entry with p > 0
+      uint32_t c = 0;
+      for (int e = tid; e < n; e += nt) c += pmass(key_at(e), kmax, smax) > 0.0 ? 1u : 0u;
+      c = static_cast<uint32_t>(block_reduce<int>(static_cast<int>(c), sh.wred_i,
+                                                  [](int x, int y) { return x + y; }));
+      if (tid == 0) sh.npos = c;
+      cl.sync();
+      int tot = 0;
+      for (int r = 0; r < C; ++r) tot += static_cast<int>(*cl.map_shared_rank(&sh.npos, r));
+      mode = VS_SELECT_TOPK;
+      k_target = min(max(tot, 1), a.k_or_cap);
+    } else {
+      double z = 0.0;
+      for (int e = tid; e < n; e += nt) z += pmass(key_at(e), kmax, smax);
+      z = block_reduce<double>(z, sh.wred_d, [](double x, double y) { return x + y; });
+      if (tid == 0) sh.zpart = z;
+      cl.sync();
+      double Z = 0.0;
+      for (int r = 0; r < C; ++r) Z += *cl.map_shared_rank(&sh.zpart, r);
+      target = a.tau * Z;
+    }
+  }
+
+  // ---- radix search for the boundary key
+  uint32_t prefix = 0, pmask = 0, cabove = 0, eqcnt = 0;
+  double mabove = 0.0;
+  int buf = 0;
+  bool by_mass = (mode == VS_SELECT_THRESHOLD);
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    prefix = 0;
+    pmask = 0;
+    cabove = 0;
+    mabove = 0.0;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      if (tid < 256) {
+        sh.cnt[buf][tid] = 0;
+        sh.mass[buf][tid] = 0.0;
+      }
+      __syncthreads();
+      for (int e = tid; e < n; e += nt) {
+        const uint32_t k = key_at(e);
+        if ((k & pmask) == prefix) {
+          const int dg = (k >> shift) & 255;
+          atomicAdd(&sh.cnt[buf][dg], 1u);
+          if (by_mass) atomicAdd(&sh.mass[buf][dg], pmass(k, kmax, smax));
+        }
+      }
+      cl.sync();
+      if (tid < 256) {
+        uint32_t c = 0;
+        double m = 0.0;
+        for (int r = 0; r < C; ++r) {
+          c += cl.map_shared_rank(&sh.cnt[buf][0], r)[tid];
+          if (by_mass) m += cl.map_shared_rank(&sh.mass[buf][0], r)[tid];
+        }
+        sh.tot_c[tid] = c;
+        sh.tot_m[tid] = m;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int bs = -1, last_nonempty = -1;
+        uint32_t ca = cabove;
+        double ma = mabove;
+        for (int b = 255; b >= 0; --b) {
+          const uint32_t c = sh.tot_c[b];
+          if (c == 0) continue;
+          last_nonempty = b;
+          if (by_mass ? (ma + sh.tot_m[b] >= target) : (ca + c >= (uint32_t)k_target)) {
+            bs = b;
+            break;
+          }
+          ca += c;
+          ma += sh.tot_m[b];
+        }
+        if (bs < 0) {  // rounding left the total just short: take the last group
+          bs = last_nonempty;
+          ca -= sh.tot_c[bs];
+          ma -= sh.tot_m[bs];
+        }
+        sh.bstar = bs;
+        sh.cabove = ca;
+        sh.mabove = ma;
+        sh.eqcnt = sh.tot_c[bs];
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(sh.bstar) << shift;
+      pmask |= 255u << shift;
+      cabove = sh.cabove;
+      mabove = sh.mabove;
+      eqcnt = sh.eqcnt;
+      buf ^= 1;
+    }
+    if (by_mass) {
+      const double pstar = pmass(prefix, kmax, smax);
+      const double need = target - mabove;
+      double mm = pstar > 0.0 ? ceil(need / pstar) : static_cast<double>(eqcnt);
+      mm = fmin(fmax(mm, 1.0), static_cast<double>(eqcnt));
+      const int k = static_cast<int>(cabove) + static_cast<int>(mm);
+      if (k > a.k_or_cap) {  // cap binds: keep the top k_or_cap instead
+        by_mass = false;
+        k_target = a.k_or_cap;
+        continue;
+      }
+      k_target = k;
+    }
+    break;
+  }
+  const uint32_t T = prefix;
+  const int m_eq = k_target - static_cast<int>(cabove);  // equal keys to keep (smallest indices)
+
+  // ---- ascending compaction across the cluster
+  const int per = (n + nt - 1) / nt;
+  const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
+  int g = 0, q = 0;
+  for (int e = e0; e < e1; ++e) {
+    const uint32_t k = key_at(e);
+    g += k > T;
+    q += k == T;
+  }
+  const int G = block_excl_scan(g, sh.scan_a);
+  const int E = block_excl_scan(q, sh.scan_b);
+  if (tid == nt - 1) {
+    sh.gt = static_cast<uint32_t>(G + g);
+    sh.eq = static_cast<uint32_t>(E + q);
+  }
+  cl.sync();
+  int eq_before = 0, sel_before = 0;
+  for (int r = 0; r < rank; ++r) {
+    const int gr = static_cast<int>(*cl.map_shared_rank(&sh.gt, r));
+    const int er = static_cast<int>(*cl.map_shared_rank(&sh.eq, r));
+    sel_before += gr + min(er, max(0, m_eq - eq_before));
+    eq_before += er;
+  }
+  int32_t* out = a.idx + (int64_t)h * a.ld_idx;
+  int pos = sel_before + G + min(E, max(0, m_eq - eq_before));
+  int eq_seen = eq_before + E;
+  for (int e = e0; e < e1; ++e) {
+    const uint32_t k = key_at(e);
+    if (k > T) {
+      out[pos++] = lo + e;
+    } else if (k == T) {
+      if (eq_seen < m_eq) out[pos++] = lo + e;
+      ++eq_seen;
+    }
+  }
+  // pad [k, k_or_cap) with -1, split over the cluster
+  for (int64_t t = (int64_t)k_target + rank * nt + tid; t < a.k_or_cap; t += (int64_t)C * nt) out[t] = -1;
+  if (rank == 0 && tid == 0) a.count[h] = k_target;
+  cl.sync();  // keep shared memory alive until every remote read is done
+}
+
+cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,
+                          double tau, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
+                          cudaStream_t stream) {
+  int C = (N + 4095) / 4096;
+  C = C < 1 ? 1 : (C > kSelMaxCluster ? kSelMaxCluster : C);
+  const int chunk = (N + C - 1) / C;
+  const bool cache = chunk <= kSelCacheKeys;
+  SelArgs a{scores, N, ld, mode, k_or_cap, tau, idx, ld_idx, count, status, chunk};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, H, 1);
+  cfg.blockDim = dim3(kSelThreads, 1, 1);
+  cfg.dynamicSmemBytes = cache ? sizeof(uint32_t) * chunk : 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (cache) {
+    e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)cfg.dynamicSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaLaunchKernelEx(&cfg, select_kernel<true>, a);
+  } else {
+    e = cudaLaunchKernelEx(&cfg, select_kernel<false>, a);
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace vs

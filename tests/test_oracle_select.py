@@ -138,3 +138,11 @@ def test_margin_detects_boundary():
     s = np.zeros(10, np.float32)
     _, cnt, margin = oracle.select(s, oracle.THRESHOLD, 10, 0.5)
     assert cnt == 5 and margin < 1e-12
+
+
+def test_margin_ignores_decisions_hidden_by_the_cap():
+    s = np.zeros(10, np.float32)
+    _, cnt, margin = oracle.select(s, oracle.THRESHOLD, 3, 0.5)  # uncapped k = 5 on a boundary
+    assert cnt == 3 and margin == np.inf
+    _, cnt, margin = oracle.select(s, oracle.THRESHOLD, 5, 0.5)  # cap == k: boundary matters
+    assert cnt == 5 and margin < 1e-12
