@@ -20,8 +20,9 @@
  *   - Every pointer argument is a DEVICE pointer on the current CUDA device
  *     (except `flags` of vs_read_device_status); the caller owns every buffer (inputs,
  *     outputs, workspace) and the stream.  The library allocates nothing,
- *     keeps no mutable global state, never writes its inputs and overwrites
- *     its outputs completely.
+ *     keeps no mutable global state (vs_sparse_attn_fwd_static_scratch is the
+ *     one documented exception), never writes its inputs and overwrites its
+ *     outputs completely.
  *   - Calls are asynchronous on `stream`; selected counts stay on the device,
  *     so select -> attention needs no host synchronisation.
  *   - Host-side argument checks run before anything is launched and return
@@ -151,6 +152,38 @@ vs_status vs_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dty
                              const int32_t* v_cnt, const int32_t* s_idx, int64_t s_ld,
                              const int32_t* s_cnt, void* O, float* lse, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * vs_sparse_attn_fwd_static_scratch -- vs_sparse_attn_fwd without a
+ * caller-provided workspace.  The summary pages have no counterpart to this
+ * call; it exists for callers that cannot allocate device memory: plain-C
+ * hosts with no device memory manager, and plug-ins inside engines that own
+ * every byte of device memory through their own pool and forbid cudaMalloc
+ * (which may also synchronise the device mid-prefill).
+ *   Same arguments and results as vs_sparse_attn_fwd, minus ws / ws_bytes;
+ *   the caller still passes every input and output buffer.
+ *   Scratch: one 16 MiB static device array inside libvs, held on every GPU
+ *   that loads the library until the process exits.  Calls needing more
+ *   (vs_attn_workspace_size(N, Hq, H_sel, d) > 16 MiB) return
+ *   VS_ERR_UNSUPPORTED before launching anything.
+ *   The first call on a device resolves the array's device address with
+ *   cudaGetSymbolAddress (with that device current); make that first call
+ *   before any stream capture.  No cudaMalloc / cudaFree or other allocating
+ *   routine is called.
+ *   Every call shares the array, which keeps the last call's contents (the
+ *   call clears what it needs to start at zero itself); calls that overlap on
+ *   the GPU -- other streams, other host threads -- race on it and must be
+ *   serialised by the caller.  The device status word of this call is not
+ *   exposed (vs_read_device_status needs a caller-owned workspace).
+ */
+vs_status vs_sparse_attn_fwd_static_scratch(const void* Q, const void* K, const void* V,
+                                            vs_dtype dtype, int N, int Hq, int Hkv, int d,
+                                            int64_t q_stride_tok, int64_t kv_stride_tok,
+                                            float softmax_scale, int H_sel, const int32_t* v_idx,
+                                            int64_t v_ld, const int32_t* v_cnt,
+                                            const int32_t* s_idx, int64_t s_ld,
+                                            const int32_t* s_cnt, void* O, float* lse,
+                                            cudaStream_t stream);
 
 /*
  * vs_dense_attn_fwd -- dense causal attention with the same kernel

@@ -39,7 +39,7 @@ VS_DEVFLAG_BOUNDS = 0x2
 EXPORTS = (
     "vs_status_string", "vs_version", "vs_index_scores", "vs_select_workspace_size", "vs_select",
     "vs_attn_workspace_size", "vs_sparse_attn_fwd", "vs_dense_attn_fwd", "vs_read_device_status",
-    "vs_selftest_wait_timeout",
+    "vs_selftest_wait_timeout", "vs_sparse_attn_fwd_static_scratch",
 )
 
 
@@ -84,6 +84,9 @@ def lib() -> ctypes.CDLL:
         L.vs_read_device_status.restype = I
         L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
         L.vs_selftest_wait_timeout.restype = I
+        L.vs_sparse_attn_fwd_static_scratch.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, I, P,
+                                                        I64, P, P, I64, P, P, P, P]
+        L.vs_sparse_attn_fwd_static_scratch.restype = I
         _lib = L
     return _lib
 
@@ -157,6 +160,19 @@ def vs_sparse_attn_fwd(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, O, lse, ws, softmax_
                                     _ptr(v_idx), v_idx.stride(0), _ptr(v_cnt), _ptr(s_idx),
                                     s_idx.stride(0), _ptr(s_cnt), _ptr(O), _ptr(lse), _ptr(ws),
                                     ws.numel(), _stream(stream)), "vs_sparse_attn_fwd")
+
+
+def vs_sparse_attn_fwd_static_scratch(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, O, lse,
+                                      softmax_scale=0.0, stream=None):
+    """vs_sparse_attn_fwd for callers that cannot allocate: uses the library's 16 MiB static
+    device scratch instead of a workspace (see include/vs_prefill.h for its limits)."""
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    _check(lib().vs_sparse_attn_fwd_static_scratch(
+        _ptr(Q), _ptr(K), _ptr(V), _dtype(Q), N, Hq, Hkv, d, Q.stride(0), K.stride(0),
+        float(softmax_scale), v_idx.shape[0], _ptr(v_idx), v_idx.stride(0), _ptr(v_cnt),
+        _ptr(s_idx), s_idx.stride(0), _ptr(s_cnt), _ptr(O), _ptr(lse), _stream(stream)),
+        "vs_sparse_attn_fwd_static_scratch")
 
 
 def vs_dense_attn_fwd(Q, K, V, O, lse, ws, softmax_scale=0.0, stream=None):
