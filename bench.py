@@ -110,6 +110,12 @@ class ClockSampler:
                 stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        # wait (up to 5 s) for the first sample so the timed region is covered
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 5:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
         return self
 
     def __exit__(self, *a):

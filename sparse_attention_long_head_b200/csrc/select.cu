@@ -188,13 +188,41 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
         sh.mass[buf][tid] = 0.0;
       }
       __syncthreads();
+      // Run-length aggregation: most keys of a pass often share one bucket, so
+      // each thread accumulates while its bucket repeats and flushes on change;
+      // the final flush is reduced across the warp when all lanes agree.
+      int cur = -1;
+      uint32_t rc = 0;
+      double rm = 0.0;
       for (int e = tid; e < n; e += nt) {
         const uint32_t k = key_at(e);
         if ((k & pmask) == prefix) {
           const int dg = (k >> shift) & 255;
-          atomicAdd(&sh.cnt[buf][dg], 1u);
-          if (by_mass) atomicAdd(&sh.mass[buf][dg], pmass(k, kmax, smax));
+          if (dg != cur) {
+            if (cur >= 0) {
+              atomicAdd(&sh.cnt[buf][cur], rc);
+              if (by_mass) atomicAdd(&sh.mass[buf][cur], rm);
+            }
+            cur = dg;
+            rc = 0;
+            rm = 0.0;
+          }
+          ++rc;
+          if (by_mass) rm += pmass(k, kmax, smax);
         }
+      }
+      __syncwarp();
+      const int cur0 = __shfl_sync(0xffffffffu, cur, 0);
+      if (__all_sync(0xffffffffu, cur == cur0) && cur0 >= 0) {
+        rc = __reduce_add_sync(0xffffffffu, rc);
+        for (int o = 16; o > 0; o >>= 1) rm += __shfl_xor_sync(0xffffffffu, rm, o);
+        if ((tid & 31) == 0) {
+          atomicAdd(&sh.cnt[buf][cur0], rc);
+          if (by_mass) atomicAdd(&sh.mass[buf][cur0], rm);
+        }
+      } else if (cur >= 0) {
+        atomicAdd(&sh.cnt[buf][cur], rc);
+        if (by_mass) atomicAdd(&sh.mass[buf][cur], rm);
       }
       cl.sync();
       if (tid < 256) {
