@@ -350,6 +350,70 @@ __device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& u
   return true;
 }
 
+// 2^x on the FMA pipe for a pair of lanes: k = round(x) via the 1.5 * 2^23
+// shifter, f = x - k in [-1/2, 1/2], 2^f by a degree-3 polynomial
+// (coefficients from csrc/fit_exp2_poly.py, max relative error 7.5e-5), and
+// 2^k added to the exponent field.  x is clamped to >= -125 so the exponent
+// stays normal; callers zero masked lanes themselves.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f,
+                  kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Which column pairs of a 128-column row take the FMA-pipe exp2 (the rest use
+// MUFU.EX2): kPolyNum out of every kPolyDen pairs.
+#ifndef VS_POLY_NUM
+#define VS_POLY_NUM 0
+#endif
+#ifndef VS_POLY_DEN
+#define VS_POLY_DEN 8
+#endif
+__host__ __device__ constexpr bool poly_pair(int j) { return (j % VS_POLY_DEN) < VS_POLY_NUM; }
+
+// p = 2^(s * scale_log2 - m) for one 128-column row (s is already -inf where
+// masked), packed to bf16 pairs into pk, row sum into ls.  One call site only:
+// two inlined copies make the compiler spill the row.
+__device__ __forceinline__ void exp_tile(const uint32_t (&sr)[4][32], const uint32_t (&mw)[4],
+                                         bool masked, float sl2, float m_base,
+                                         uint32_t (&pk)[2][32], float& ls) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+      const float x0 = fmaf(__uint_as_float(sr[q][c]), sl2, -m_base);
+      const float x1 = fmaf(__uint_as_float(sr[q][c + 1]), sl2, -m_base);
+      float p0, p1;
+      if (poly_pair(q * 16 + c / 2)) {
+        const float2 pp = exp2_fma2(make_float2(x0, x1));
+        p0 = pp.x;
+        p1 = pp.y;
+        if (masked) {
+          if (!((mw[q] >> c) & 1u)) p0 = 0.f;
+          if (!((mw[q] >> (c + 1)) & 1u)) p1 = 0.f;
+        }
+      } else {
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      acc[(c >> 1) & 1] += p0;
+      acc[2 + ((c >> 1) & 1)] += p1;
+      pk[q >> 1][(q & 1) * 16 + c / 2] = pack_bf16x2(p0, p1);
+    }
+  }
+  ls = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 template <int D, bool SPARSE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -444,17 +508,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         reg_pin(sr[1]);
         reg_pin(sr[2]);
         reg_pin(sr[3]);
-        float mx = -INFINITY;
+        if (masked) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float v = __uint_as_float(sr[q][c]);
-            if (masked && !((mw[q] >> c) & 1u)) v = -INFINITY;
-            sr[q][c] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
-          }
+            for (int c = 0; c < 32; ++c)
+              if (!((mw[q] >> c) & 1u)) sr[q][c] = __float_as_uint(-INFINITY);
         }
+        // row max: eight independent chains of three-input max
+        float m8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) m8[t] = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int c = 0; c < 32; c += 2)
+            m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], __uint_as_float(sr[q][c]),
+                                     __uint_as_float(sr[q][c + 1]));
+        const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]),
+                               fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
         const float m_cand = mx * P.scale_log2;
         const bool need = m_cand > m_use + 8.0f;
         float factor = 1.f;
@@ -466,20 +538,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float m_base = m_use == -INFINITY ? 0.f : m_use;
         float ls = 0.f;
         uint32_t pk[2][32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][c]), P.scale_log2, -m_base));
-            float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][c + 1]), P.scale_log2, -m_base));
-            ls += p0 + p1;
-            pk[q >> 1][(q & 1) * 16 + c / 2] = pack_bf16x2(p0, p1);
-          }
-        }
+        exp_tile(sr, mw, masked, P.scale_log2, m_base, pk, ls);
         l += ls;
         tmem_st32(tS, pk[0]);
         tmem_st32(tS + 32, pk[1]);
         if (k > 0 && __any_sync(0xffffffffu, need)) {
+          // O must be rescaled before PV(k) accumulates into it; PV(k-1) is
+          // complete because S(k) was issued after it.
 #pragma unroll 1
           for (int q = 0; q < D / 32; ++q) {
             uint32_t o[32];
@@ -530,22 +595,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t q_addr = smem_u32(sQ), kv_addr = smem_u32(sKV);
       uint32_t seq = 0, ucount = 0, pcnt[2] = {0, 0};
       bool ok = true;
+      // Descriptors of the tile bases; per-MMA k offsets are compile-time
+      // constants added to the 14-bit start-address field (addresses < 256 KB,
+      // so the field never carries into its neighbour).
+      const uint64_t qdesc = sdesc_sw128(q_addr, 16, 1024);
+      const uint64_t kdesc = sdesc_sw128(kv_addr, 16, 1024);
+      const uint64_t vdesc = sdesc_sw128(kv_addr, 16384, 1024);
       auto issue_s = [&](int sub, uint32_t slot) {
+        const uint64_t ad = qdesc + ((sub * C::kQBytes) >> 4);
+        const uint64_t bd = kdesc + ((slot * C::kTileBytes) >> 4);
+        const uint32_t d = tbase + sub * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(q_addr + sub * C::kQBytes + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kv_addr + slot * C::kTileBytes + off, 16, 1024);
-          mma_ss(tbase + sub * 128, ad, bd, idesc_qk, kk > 0);
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_ss(d, ad + off, bd + off, idesc_qk, kk > 0);
         }
       };
       auto issue_pv = [&](int sub, uint32_t slot, bool acc) {
+        const uint64_t bd = vdesc + ((slot * C::kTileBytes) >> 4);
+        const uint32_t d = tbase + 256 + sub * 128, a = tbase + sub * 128;
+        mma_ts(d, a, bd, idesc_pv, acc ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = sdesc_sw128(kv_addr + slot * C::kTileBytes + kk * 2048, 16384, 1024);
-          mma_ts(tbase + 256 + sub * 128, tbase + sub * 128 + kk * 8, bd, idesc_pv,
-                 (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 1; kk < 8; ++kk) mma_ts(d, a + kk * 8, bd + ((kk * 2048) >> 4), idesc_pv, 1u);
       };
       for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
         const UnitInfo ui = unit_info<SPARSE>(P, u);
@@ -564,6 +635,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t vslot = seq % S;
           if (!mbar_wait(bar(B_FULL + vslot), (seq / S) & 1, wc)) { ok = false; break; }
           ++seq;
+          if (k + 1 < ui.n) {  // next K tile, waited for off the critical path
+            kslot = seq % S;
+            if (!mbar_wait(bar(B_FULL + kslot), (seq / S) & 1, wc)) { ok = false; break; }
+            ++seq;
+          }
           for (int sub = 0; sub < 2; ++sub) {
             if (!mbar_wait(bar(B_PFULL + sub), pcnt[sub] & 1, wc)) { ok = false; break; }
             ++pcnt[sub];
@@ -574,12 +650,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             issue_pv(sub, vslot, k > 0);
             if (sub == 1) mma_commit(bar(B_EMPTY + vslot));
             if (k + 1 < ui.n) {
-              if (sub == 0) {
-                kslot = seq % S;
-                if (!mbar_wait(bar(B_FULL + kslot), (seq / S) & 1, wc)) { ok = false; break; }
-                ++seq;
-                tc_fence_after();
-              }
               issue_s(sub, kslot);
               mma_commit(bar(B_SFULL + sub));
               if (sub == 1) mma_commit(bar(B_EMPTY + kslot));
