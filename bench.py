@@ -157,17 +157,25 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def kernel_rev() -> str:
+    """Hash of the attention kernel sources: a committed traffic figure is only
+    used while the kernel it was measured on is unchanged."""
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("attn_tc.cu", "ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "sparse_attention_long_head_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
 def ncu_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    """DRAM bytes (read + write) per attention launch from the committed ncu
+    summary for this workload, or None if absent or taken on another kernel."""
+    p = os.path.join(ROOT, "profiles", f"attn_traffic_{workload}.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        if d.get("workload") == workload and d.get("kernel_rev") == KERNEL_REV:
+        if d.get("kernel_rev") == kernel_rev():
             return d.get("dram_bytes_per_launch")
     return None
-
-
-KERNEL_REV = "attn_tc_v1"
 
 
 # --------------------------------------------------------------- our arm
@@ -423,7 +431,8 @@ def _cpu_cores():
         return os.cpu_count()
 
 
-def cpu_baseline(w, Qb, Kb, Vb, vi, vc, si, sc, seconds, seed=0):
+def cpu_baseline(w, Qb, Kb, Vb, vi, vc, si, sc, seconds, seed=0,
+                 sets_from="this run's GPU selection"):
     """The fp64 oracle as it stands, timed on a bounded row sample of the same
     workload; scaled to the metric by pair count (oracle effective TFLOP/s)."""
     import oracle
@@ -448,7 +457,7 @@ def cpu_baseline(w, Qb, Kb, Vb, vi, vc, si, sc, seconds, seed=0):
             "kind": "oracle",
             "sample": f"{rows_done} query rows (32 random rows of a random head per draw, "
                       f"{len(set(heads))} heads) of {w.name}, fp64 row-form oracle with OpenMP over "
-                      f"rows, {t_used:.1f} s; index sets from this run's GPU selection"}
+                      f"rows, {t_used:.1f} s; index sets from {sets_from}"}
 
 
 def run_reference(args, w):
@@ -473,7 +482,8 @@ def run_reference(args, w):
     vals = []
     last = None
     for it in range(args.warmup + args.steps):
-        last = cpu_baseline(w, Qb, Kb, Vb, vi, vc, si, sc, per_step, seed=it)
+        last = cpu_baseline(w, Qb, Kb, Vb, vi, vc, si, sc, per_step, seed=it,
+                            sets_from="the oracle's own selection")
         if it >= args.warmup:
             vals.append(last["value"])
     value = float(np.mean(vals))

@@ -10,7 +10,8 @@
 //     offsets), an ascending column list, and the list of touched
 //     block-diagonals.  No n x n structure is ever built.
 //   * The attention kernel is persistent: one CTA per SM walks "units" of 256
-//     query rows of one head (two 128-row sub-tiles A and B), heaviest first.
+//     query rows of one head (two 128-row sub-tiles A and B), KV head by KV
+//     head (L2 reuse of K/V), heaviest first within a KV head.
 //   * Per unit it streams "items": 128-key blocks loaded by TMA (tiled), or
 //     128-column chunks of the vertical list gathered row by row with TMA
 //     tile::gather4.  Each item is applied to both sub-tiles.
@@ -235,10 +236,14 @@ struct UnitInfo {
 
 template <bool SPARSE>
 __device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
+  // Units grouped by KV head (so CTAs running at the same time stream the same
+  // K/V and share it in L2), heaviest (largest p) first within a group, the G
+  // query heads of a group adjacent.
   UnitInfo ui;
-  ui.p = P.P - 1 - u / P.Hq;
-  ui.h = u % P.Hq;
-  ui.g = ui.h / P.G;
+  ui.g = u / (P.G * P.P);
+  const int rem = u - ui.g * P.G * P.P;
+  ui.p = P.P - 1 - rem / P.G;
+  ui.h = ui.g * P.G + rem % P.G;
   ui.hs = (int)(((int64_t)ui.h * P.H_sel) / P.Hq);
   const int last_b = min(2 * ui.p + 1, P.T - 1);
   const int n_dense = last_b + 1;
