@@ -87,6 +87,32 @@ def total_pairs(N, Hq, vi, vc, si, sc):
     return sum(per[(h * H_sel) // Hq] for h in range(Hq)), per
 
 
+# ----------------------------------------------------------- multi-rank
+
+
+def dist_env():
+    """(world, rank, local_rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity at world 1)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_value(world: int, flops_per_rank: float, ms: float) -> float:
+    """Aggregate effective TFLOP/s: every rank processes one replica of the layer in
+    (at most) `ms`, so the job does world x flops in that time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- clocks
 
 
@@ -187,9 +213,7 @@ def run_ours(args, w):
 
     import sparse_attention_long_head_b200 as vs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
@@ -286,11 +310,8 @@ def run_ours(args, w):
     ms_step = float(np.mean(step_ms))
     ms_att = float(np.mean(att_ms))
     ms_sel = float(np.mean(sel_ms))
-    if world > 1:
-        t = torch.tensor([ms_step, ms_att], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, ms_att = float(t[0]), float(t[1])
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    ms_step, ms_att = max_over_ranks([ms_step, ms_att], dev)
+    value = whole_job_value(world, flops, ms_step)
 
     # dense causal kernel on the same inputs (speed-up denominator)
     ws_dense = vs.workspace(256, dev)
@@ -339,12 +360,8 @@ def run_ours(args, w):
             b.record(stream)
             b.synchronize()
             ts.append(a.elapsed_time(b))
-        e2e_ms = float(np.min(ts[1:] if len(ts) > 1 else ts))
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t[0])
-        e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        e2e_ms = max_over_ranks([float(np.min(ts[1:] if len(ts) > 1 else ts))], dev)[0]
+        e2e = {"value": round(whole_job_value(world, flops, e2e_ms), 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
@@ -462,8 +479,7 @@ def cpu_baseline(w, Qb, Kb, Vb, vi, vc, si, sc, seconds, seed=0,
 
 def run_reference(args, w):
     """Reference arm: the oracle as it stands on the host cores, rank 0 only."""
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    world, rank, _ = dist_env()
     if rank != 0:
         return
     import oracle
