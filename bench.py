@@ -252,7 +252,7 @@ def run_ours(args, w):
     lse = torch.empty((Hq, N), dtype=torch.float32, device=dev)
     ws_sel = vs.workspace(vs.vs_select_workspace_size(H_sel, N), dev)
     ws_sel2 = vs.workspace(vs.vs_select_workspace_size(H_sel, N), dev)
-    ws_att = vs.workspace(vs.vs_attn_workspace_size(N, Hq, H_sel, d), dev)
+    ws_att = vs.workspace(vs.vs_attn_workspace_size_ld(N, Hq, H_sel, d, w.k_v), dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     launches_per_step = 4 + (1 if w.indexer else 0)
 

@@ -142,10 +142,16 @@ vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_sel
  *            cnt entries of each row used; duplicates and order do not matter).
  *   O        [N, Hq, d] in `dtype` with token stride q_stride_tok (output).
  *   lse      fp32 [Hq][N] (output) or NULL.
- *   ws       device workspace, >= vs_attn_workspace_size(N, Hq, H_sel, d)
- *            bytes, 256-byte aligned.
+ *   ws       device workspace, 256-byte aligned, of at least
+ *            vs_attn_workspace_size(N, Hq, H_sel, d) bytes (the plan).  With
+ *            vs_attn_workspace_size_ld(N, Hq, H_sel, d, v_ld) bytes or more the
+ *            selected vertical K/V rows are first packed contiguously and then
+ *            loaded as tiles (when every index set's query heads lie in one KV
+ *            group); with less they are gathered row by row.  Results are the
+ *            same either way.
  */
 size_t vs_attn_workspace_size(int N, int Hq, int H_sel, int d);
+size_t vs_attn_workspace_size_ld(int N, int Hq, int H_sel, int d, int64_t v_ld);
 vs_status vs_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
                              int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
                              float softmax_scale, int H_sel, const int32_t* v_idx, int64_t v_ld,

@@ -39,7 +39,7 @@ VS_DEVFLAG_BOUNDS = 0x2
 EXPORTS = (
     "vs_status_string", "vs_version", "vs_index_scores", "vs_select_workspace_size", "vs_select",
     "vs_attn_workspace_size", "vs_sparse_attn_fwd", "vs_dense_attn_fwd", "vs_read_device_status",
-    "vs_selftest_wait_timeout", "vs_sparse_attn_fwd_static_scratch",
+    "vs_selftest_wait_timeout", "vs_sparse_attn_fwd_static_scratch", "vs_attn_workspace_size_ld",
 )
 
 
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.vs_select.restype = I
         L.vs_attn_workspace_size.argtypes = [I, I, I, I]
         L.vs_attn_workspace_size.restype = Z
+        L.vs_attn_workspace_size_ld.argtypes = [I, I, I, I, I64]
+        L.vs_attn_workspace_size_ld.restype = Z
         L.vs_sparse_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, I, P, I64, P, P, I64,
                                          P, P, P, P, Z, P]
         L.vs_sparse_attn_fwd.restype = I
@@ -130,6 +132,10 @@ def vs_select_workspace_size(H: int, N: int) -> int:
 
 def vs_attn_workspace_size(N: int, Hq: int, H_sel: int, d: int) -> int:
     return lib().vs_attn_workspace_size(N, Hq, H_sel, d)
+
+
+def vs_attn_workspace_size_ld(N: int, Hq: int, H_sel: int, d: int, v_ld: int) -> int:
+    return lib().vs_attn_workspace_size_ld(N, Hq, H_sel, d, v_ld)
 
 
 def vs_index_scores(K, V, W1, W2, logits_v, logits_s, stream=None):
@@ -219,7 +225,8 @@ def sparse_attention(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, ws=None, with_lse=True
     O = torch.empty_like(Q)
     lse = torch.empty((Hq, N), dtype=torch.float32, device=Q.device) if with_lse else None
     if ws is None:
-        ws = workspace(vs_attn_workspace_size(N, Hq, v_idx.shape[0], d), Q.device)
+        ws = workspace(vs_attn_workspace_size_ld(N, Hq, v_idx.shape[0], d, v_idx.stride(0)),
+                       Q.device)
     vs_sparse_attn_fwd(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, O, lse, ws, stream=stream)
     return O, lse
 

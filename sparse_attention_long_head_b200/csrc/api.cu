@@ -129,6 +129,14 @@ vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_sel
   return VS_OK;
 }
 
+size_t vs_attn_workspace_size_ld(int N, int Hq, int H_sel, int d, int64_t v_ld) {
+  (void)Hq;
+  if (N < 1 || H_sel < 1 || (d != 64 && d != 128) || v_ld < 1) return kStatusBytes;
+  const PlanLayout L = PlanLayout::make(N, H_sel);
+  const PackedLayout Pk = PackedLayout::make(L, H_sel, d, v_ld);
+  return Pk.offset + Pk.bytes;
+}
+
 size_t vs_attn_workspace_size(int N, int Hq, int H_sel, int d) {
   (void)Hq;
   (void)d;
@@ -152,7 +160,8 @@ static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype
   } else {
     H_sel = 1;
   }
-  const size_t need = sparse ? vs_attn_workspace_size(N, Hq, H_sel, d) : kStatusBytes;
+  const PlanLayout L = PlanLayout::make(N, H_sel);
+  const size_t need = sparse ? L.total : kStatusBytes;  // the plan alone suffices
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
   AttnArgs a;
   a.Q = Q;
@@ -178,9 +187,19 @@ static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype
   a.ws = ws;
   a.status = static_cast<int*>(ws);
   a.stream = stream;
-  const PlanLayout L = PlanLayout::make(N, H_sel);
+  a.pack_vrows = 0;
+  a.pack_k = a.pack_v = nullptr;
+  if (sparse && dtype == VS_BF16 && PackedLayout::eligible(Hq, Hkv, H_sel)) {
+    const PackedLayout Pk = PackedLayout::make(L, H_sel, d, v_ld);
+    if (ws_bytes >= Pk.offset + Pk.bytes) {  // room to pack the vertical rows
+      a.pack_vrows = Pk.vrows;
+      a.pack_k = static_cast<char*>(ws) + Pk.offset;
+      a.pack_v = static_cast<char*>(ws) + Pk.offset + Pk.bytes / 2;
+    }
+  }
   if (cudaMemsetAsync(a.status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
   if (sparse && launch_plan(a, L) != cudaSuccess) return VS_ERR_CUDA;
+  if (a.pack_vrows > 0 && launch_pack(a, L) != cudaSuccess) return VS_ERR_CUDA;
   cudaError_t e = dtype == VS_BF16 ? launch_attn_tc(a, L) : launch_attn_fp32(a, L);
   return e == cudaSuccess ? VS_OK : VS_ERR_CUDA;
 }

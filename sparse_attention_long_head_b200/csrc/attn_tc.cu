@@ -13,8 +13,10 @@
 //     query rows of one head (two 128-row sub-tiles A and B), KV head by KV
 //     head (L2 reuse of K/V), heaviest first within a KV head.
 //   * Per unit it streams "items": 128-key blocks loaded by TMA (tiled), or
-//     128-column chunks of the vertical list gathered row by row with TMA
-//     tile::gather4.  Each item is applied to both sub-tiles.
+//     128-column chunks of the vertical list -- as tiles of the packed copy a
+//     pack kernel writes before the attention kernel, or, when the workspace
+//     has no room for it, gathered row by row with TMA tile::gather4.  Each
+//     item is applied to both sub-tiles.
 //   * QK^T and PV run on tcgen05 (bf16 in, fp32 accumulate in TMEM); P is
 //     written back into TMEM over S and consumed by the TS-form MMA.
 //   * Four softmax warps per sub-tile own one row each; the element mask of a
@@ -198,6 +200,53 @@ cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ pack
+
+// Copies each index set's selected K and V rows (ascending column order) into
+// [H_sel][vrows][d] buffers, zero-filling the rest of the last 128-row chunk.
+// One CTA per (128-row chunk, index set); chunks past the set's count exit.
+template <int D>
+__global__ void __launch_bounds__(256) pack_kernel(const __nv_bfloat16* K, const __nv_bfloat16* V,
+                                                   int64_t kv_stride, int Hq, int Hkv, int H_sel,
+                                                   int64_t vrows, PlanLayout L, PlanPtrs pp,
+                                                   __nv_bfloat16* pk, __nv_bfloat16* pv) {
+  const int hs = blockIdx.y, c = blockIdx.x;
+  const int nv = pp.meta[4 * hs + 0];
+  if (128 * c >= nv) return;
+  const int g = (hs * (Hq / H_sel)) / (Hq / Hkv);
+  const int32_t* vl = pp.vlist + (int64_t)hs * L.N;
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  for (int e = threadIdx.x; e < 128 * CH; e += blockDim.x) {
+    const int r = e / CH, ch = e % CH;
+    const int t = 128 * c + r;
+    uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (t < nv) {
+      const int64_t src = (int64_t)vl[t] * kv_stride + (int64_t)g * D + ch * 8;
+      kk = *reinterpret_cast<const uint4*>(K + src);
+      vv = *reinterpret_cast<const uint4*>(V + src);
+    }
+    const int64_t dst = ((int64_t)hs * vrows + t) * D + ch * 8;
+    *reinterpret_cast<uint4*>(pk + dst) = kk;
+    *reinterpret_cast<uint4*>(pv + dst) = vv;
+  }
+}
+
+cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L) {
+  dim3 grid((unsigned)(a.pack_vrows / 128), (unsigned)a.H_sel);
+  const PlanPtrs pp = plan_ptrs(L, a.ws);
+  auto* K = static_cast<const __nv_bfloat16*>(a.K);
+  auto* V = static_cast<const __nv_bfloat16*>(a.V);
+  auto* pk = static_cast<__nv_bfloat16*>(a.pack_k);
+  auto* pv = static_cast<__nv_bfloat16*>(a.pack_v);
+  if (a.d == 128)
+    pack_kernel<128><<<grid, 256, 0, a.stream>>>(K, V, a.kv_stride, a.Hq, a.Hkv, a.H_sel,
+                                                 a.pack_vrows, L, pp, pk, pv);
+  else
+    pack_kernel<64><<<grid, 256, 0, a.stream>>>(K, V, a.kv_stride, a.Hq, a.Hkv, a.H_sel,
+                                                a.pack_vrows, L, pp, pk, pv);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------- attention
 
 constexpr int kAttnThreads = 320;
@@ -228,6 +277,7 @@ struct AttnParams {
   uint64_t wait_limit_ns;
   PlanLayout L;
   PlanPtrs pp;
+  int64_t pack_vrows;  // 0: gather vertical rows; else packed tiles (tmKg/tmVg map them)
 };
 
 struct UnitInfo {
@@ -706,6 +756,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int h = 0; h < nsub64; ++h)
                 tma_load_2d(dst + h * 16384, m, fb, ui.g * D + 64 * h, 128 * it.b);
             }
+          } else if (P.pack_vrows > 0) {
+            if (lane == 0) {
+              const CUtensorMap* m = kv ? &tmVg : &tmKg;
+              for (int h = 0; h < nsub64; ++h)
+                tma_load_2d(dst + h * 16384, m, fb, 64 * h,
+                            (int)(ui.hs * P.pack_vrows + 128 * it.b));
+            }
           } else {
             const int32_t* base = P.pp.vlist + (int64_t)ui.hs * P.N + 128 * it.b;
             const int cnt = min(128, ui.nv - 128 * it.b);
@@ -764,8 +821,13 @@ static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
   encode_map(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.N, a.q_stride, 128, &rc);
   encode_map(enc, &mK, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, 128, &rc);
   encode_map(enc, &mV, a.V, (int64_t)a.Hkv * D, a.N, a.kv_stride, 128, &rc);
-  encode_map(enc, &mKg, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
-  encode_map(enc, &mVg, a.V, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
+  if (SPARSE && a.pack_vrows > 0) {  // packed vertical rows: [H_sel * vrows][D] tiles
+    encode_map(enc, &mKg, a.pack_k, D, (int64_t)a.H_sel * a.pack_vrows, D, 128, &rc);
+    encode_map(enc, &mVg, a.pack_v, D, (int64_t)a.H_sel * a.pack_vrows, D, 128, &rc);
+  } else {
+    encode_map(enc, &mKg, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
+    encode_map(enc, &mVg, a.V, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
+  }
   if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
   AttnParams P;
   P.N = a.N;
@@ -784,6 +846,7 @@ static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
   P.wait_limit_ns = kDefaultWaitLimitNs;
   P.L = L;
   P.pp = plan_ptrs(L, a.ws);
+  P.pack_vrows = SPARSE ? a.pack_vrows : 0;
   auto kern = attn_tc_kernel<D, SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg<D>::kSmem);

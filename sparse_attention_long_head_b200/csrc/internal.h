@@ -95,6 +95,28 @@ inline __host__ __device__ PlanPtrs plan_ptrs(const PlanLayout& L, void* ws) {
   return p;
 }
 
+// Optional region after the plan: each index set's selected vertical K and V
+// rows packed contiguously ([H_sel][vrows][d] each), so that vertical chunks
+// load as ordinary TMA tiles instead of row gathers.  Used when every index
+// set's query heads lie in one KV group ((Hq / H_sel) divides Hq / Hkv) and the
+// workspace is large enough.
+struct PackedLayout {
+  int64_t vrows = 0;  // rows per index set, multiple of 128
+  size_t offset = 0, bytes = 0;
+  static bool eligible(int Hq, int Hkv, int H_sel) {
+    const int qs = Hq / H_sel, G = Hq / Hkv;
+    return qs >= 1 && G % qs == 0;
+  }
+  static PackedLayout make(const PlanLayout& L, int H_sel, int d, int64_t v_ld) {
+    PackedLayout Pk;
+    const int64_t rows = v_ld < L.N ? v_ld : L.N;
+    Pk.vrows = (rows + 127) / 128 * 128;
+    Pk.offset = (L.total + 1023) / 1024 * 1024;
+    Pk.bytes = 2 * (size_t)H_sel * (size_t)Pk.vrows * (size_t)d * 2;
+    return Pk;
+  }
+};
+
 // Common attention launch description.
 struct AttnArgs {
   const void* Q;
@@ -115,10 +137,15 @@ struct AttnArgs {
   void* ws;
   int* status;
   cudaStream_t stream;
+  // packed vertical rows (vrows == 0: gather the rows with TMA gather4)
+  int64_t pack_vrows;
+  void* pack_k;
+  void* pack_v;
 };
 
 // Launchers (return a CUDA error; argument checks are done by the caller).
 cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L);
+cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_attn_tc(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_attn_fp32(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,

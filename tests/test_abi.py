@@ -47,6 +47,10 @@ def test_workspace_sizes():
     assert 256 < small < big
     # plan data is O(N) per index-set head: bitmaps + lists, no N x N structure
     assert big < 8 * 262144 * 4 * 4
+    # room to pack the selected vertical K/V rows: 2 x H_sel x roundup(v_ld, 128) x d x 2 bytes
+    packed = vs.vs_attn_workspace_size_ld(262144, 32, 8, 128, 16384)
+    assert packed >= big + 2 * 8 * 16384 * 128 * 2
+    assert vs.vs_attn_workspace_size_ld(1024, 1, 1, 64, 5) >= small + 2 * 128 * 64 * 2
 
 
 P = ctypes.c_void_p

@@ -180,3 +180,29 @@ def test_custom_scale_and_strided_tokens(cuda_device):
     for h in range(Hq):
         Or, lr = oracle.attn_rows(Qb, Kb, Vb, h, np.arange(N), vi, vc, si, sc, scale=0.05)
         compare_rows(Od[:, h], Or, lse[h].cpu().numpy(), lr, what=f"strided head {h}")
+
+
+def test_packed_and_gathered_vertical_paths_agree(cuda_device):
+    # same call with the plan-only workspace (row gathers) and with room to
+    # pack the vertical rows (tile loads): identical outputs
+    N, d = 3000, 128
+    rng = np.random.default_rng(21)
+    Qb, Kb, Vb = gen_qkv(22, N, 4, 2, d, 500000.0)
+    v_sets = [np.sort(rng.choice(N, n, replace=False)) for n in (700, 129, 1, 0)]
+    s_sets = [np.array([0, 1, 2]), np.arange(0, 40), np.array([0]), np.array([5, 900])]
+    vi, vc = sets_to_rows(v_sets, 1000)
+    si, sc = sets_to_rows(s_sets)
+    Q, K, V = (bf16_to_dev(x) for x in (Qb, Kb, Vb))
+    args = [torch.from_numpy(x).cuda() for x in (vi, vc, si, sc)]
+    outs = []
+    for nbytes in (vs.vs_attn_workspace_size(N, 4, 4, d),
+                   vs.vs_attn_workspace_size_ld(N, 4, 4, d, vi.shape[1])):
+        ws = vs.workspace(nbytes)
+        O, lse = vs.sparse_attention(Q, K, V, *args, ws=ws)
+        assert vs.vs_read_device_status(ws)[0] == vs.VS_OK
+        outs.append((O.clone(), lse.clone()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    Od = dev_to_f64(outs[1][0])
+    for h in range(4):
+        Or, lr = oracle.attn_rows(Qb, Kb, Vb, h, np.arange(N), vi, vc, si, sc)
+        compare_rows(Od[:, h], Or, outs[1][1][h].cpu().numpy(), lr, what=f"packed head {h}")
