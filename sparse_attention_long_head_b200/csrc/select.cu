@@ -9,16 +9,19 @@
 // (section 1) notes that sorting and cumulative sums are what make such
 // selection expensive on GPUs; this kernel therefore never sorts:
 //
-//   * One thread-block cluster per head (C <= 8 CTAs); each CTA keeps its
-//     slice of the scores as order-preserving 32-bit keys in shared memory.
-//   * A most-significant-digit radix search (4 passes of 8 bits) finds the
-//     exact boundary key.  Per pass every CTA builds a 256-bucket histogram of
-//     counts (and, for the threshold rule, of fp64 softmax mass); the cluster
+//   * One thread-block cluster per head (8 CTAs, 16 when there are few
+//     heads); each CTA keeps its slice of the scores as order-preserving
+//     32-bit keys in shared memory.
+//   * Most-significant-digit radix searches (4 passes of 8 bits) find the
+//     exact boundary keys.  Per pass every CTA builds 256-bucket histograms
+//     of counts and, for the threshold rule, of fp64 softmax mass; the cluster
 //     merges them through distributed shared memory, and every CTA takes the
 //     same decision from the same merged data.
 //   * The threshold rule walks the buckets from the top, accumulating mass
-//     until tau * Z is reached; inside the final group of equal keys the
-//     count follows from their common mass.
+//     until tau * Z is reached (Z = the total of the first pass's mass
+//     histogram); inside the final group of equal keys the count follows from
+//     their common mass.  The top-cap boundary is searched in the same passes,
+//     so a capped head needs no second search.
 //   * A last pass writes the kept indices in ascending order (index-ordered
 //     compaction across the cluster), then pads with -1.
 #include <cooperative_groups.h>
@@ -60,17 +63,17 @@ struct SelArgs {
 };
 
 struct SelShared {
-  uint32_t cnt[2][256];
-  double mass[2][256];
-  uint32_t tot_c[256];
-  double tot_m[256];
+  uint32_t cnt_c[2][256];   // count histogram of the top-k (cap) search
+  uint32_t cnt_t[2][256];   // count histogram of the threshold search
+  double mass_t[2][256];    // mass histogram of the threshold search
+  uint32_t tot_cc[256], tot_ct[256];
+  double tot_mt[256];
   uint32_t kmax;
-  double zpart;
   uint32_t npos;
   uint32_t gt, eq;
-  int bstar;
-  uint32_t cabove, eqcnt;
-  double mabove;
+  int bstar_c, bstar_t;
+  uint32_t cabove_c, cabove_t, eqcnt_t;
+  double mabove_t, target;
   int wred_i[32];
   double wred_d[32];
   int scan_a[kSelThreads];
@@ -141,13 +144,18 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   for (int r = 0; r < C; ++r) kmax = max(kmax, *cl.map_shared_rank(&sh.kmax, r));
   const double smax = static_cast<double>(fkey_inv(kmax));
 
-  int mode = a.mode;
-  int k_target = a.k_or_cap;
-  double target = 0.0;
-  if (mode == VS_SELECT_THRESHOLD) {
+  // Two most-significant-digit radix searches share the passes over the keys:
+  //   count path: the key of the k-th entry (k = the top-k budget or the cap);
+  //   mass path (threshold rule): the key where the running softmax mass in
+  //     descending order reaches tau * Z; Z is the total of pass 0's mass
+  //     histogram, so it needs no pass of its own.
+  // The threshold result is used when it keeps at most `cap` entries, else the
+  // count path's top-cap result (k = min(k_threshold, cap)).
+  int k_count = a.k_or_cap;
+  bool use_mass = false;
+  if (a.mode == VS_SELECT_THRESHOLD) {
     if (kmax == 0u) {  // every score is NaN: keep one entry
-      mode = VS_SELECT_TOPK;
-      k_target = 1;
+      k_count = 1;
     } else if (a.tau >= 1.0) {  // keep every entry with p > 0
       uint32_t c = 0;
       for (int e = tid; e < n; e += nt) c += pmass(key_at(e), kmax, smax) > 0.0 ? 1u : 0u;
@@ -157,134 +165,172 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
       cl.sync();
       int tot = 0;
       for (int r = 0; r < C; ++r) tot += static_cast<int>(*cl.map_shared_rank(&sh.npos, r));
-      mode = VS_SELECT_TOPK;
-      k_target = min(max(tot, 1), a.k_or_cap);
+      k_count = min(max(tot, 1), a.k_or_cap);
     } else {
-      double z = 0.0;
-      for (int e = tid; e < n; e += nt) z += pmass(key_at(e), kmax, smax);
-      z = block_reduce<double>(z, sh.wred_d, [](double x, double y) { return x + y; });
-      if (tid == 0) sh.zpart = z;
-      cl.sync();
-      double Z = 0.0;
-      for (int r = 0; r < C; ++r) Z += *cl.map_shared_rank(&sh.zpart, r);
-      target = a.tau * Z;
+      use_mass = true;
     }
   }
 
-  // ---- radix search for the boundary key
-  uint32_t prefix = 0, pmask = 0, cabove = 0, eqcnt = 0;
-  double mabove = 0.0;
+  uint32_t pf_c = 0, pm_c = 0, cab_c = 0;            // count path
+  uint32_t pf_t = 0, pm_t = 0, cab_t = 0, eq_t = 0;  // mass path
+  double mab_t = 0.0, target = 0.0;
   int buf = 0;
-  bool by_mass = (mode == VS_SELECT_THRESHOLD);
-  for (int attempt = 0; attempt < 2; ++attempt) {
-    prefix = 0;
-    pmask = 0;
-    cabove = 0;
-    mabove = 0.0;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      if (tid < 256) {
-        sh.cnt[buf][tid] = 0;
-        sh.mass[buf][tid] = 0.0;
-      }
-      __syncthreads();
-      // Run-length aggregation: most keys of a pass often share one bucket, so
-      // each thread accumulates while its bucket repeats and flushes on change;
-      // the final flush is reduced across the warp when all lanes agree.
-      int cur = -1;
-      uint32_t rc = 0;
-      double rm = 0.0;
-      for (int e = tid; e < n; e += nt) {
-        const uint32_t k = key_at(e);
-        if ((k & pmask) == prefix) {
-          const int dg = (k >> shift) & 255;
-          if (dg != cur) {
-            if (cur >= 0) {
-              atomicAdd(&sh.cnt[buf][cur], rc);
-              if (by_mass) atomicAdd(&sh.mass[buf][cur], rm);
-            }
-            cur = dg;
-            rc = 0;
-            rm = 0.0;
-          }
-          ++rc;
-          if (by_mass) rm += pmass(k, kmax, smax);
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    if (tid < 256) {
+      sh.cnt_c[buf][tid] = 0;
+      sh.cnt_t[buf][tid] = 0;
+      sh.mass_t[buf][tid] = 0.0;
+    }
+    __syncthreads();
+    // Run-length aggregation per search: keys of a pass often fall in one
+    // bucket, so a thread accumulates while its bucket repeats and flushes on
+    // change; the final flush is reduced across the warp when all lanes agree.
+    int cur_c = -1, cur_t = -1;
+    uint32_t rc_c = 0, rc_t = 0;
+    double rm_t = 0.0;
+    for (int e = tid; e < n; e += nt) {
+      const uint32_t k = key_at(e);
+      if ((k & pm_c) == pf_c) {
+        const int dg = (k >> shift) & 255;
+        if (dg != cur_c) {
+          if (cur_c >= 0) atomicAdd(&sh.cnt_c[buf][cur_c], rc_c);
+          cur_c = dg;
+          rc_c = 0;
         }
+        ++rc_c;
       }
-      __syncwarp();
-      const int cur0 = __shfl_sync(0xffffffffu, cur, 0);
-      if (__all_sync(0xffffffffu, cur == cur0) && cur0 >= 0) {
-        rc = __reduce_add_sync(0xffffffffu, rc);
-        for (int o = 16; o > 0; o >>= 1) rm += __shfl_xor_sync(0xffffffffu, rm, o);
+      if (use_mass && (k & pm_t) == pf_t) {
+        const int dg = (k >> shift) & 255;
+        if (dg != cur_t) {
+          if (cur_t >= 0) {
+            atomicAdd(&sh.cnt_t[buf][cur_t], rc_t);
+            atomicAdd(&sh.mass_t[buf][cur_t], rm_t);
+          }
+          cur_t = dg;
+          rc_t = 0;
+          rm_t = 0.0;
+        }
+        ++rc_t;
+        rm_t += pmass(k, kmax, smax);
+      }
+    }
+    __syncwarp();
+    {
+      const int c0 = __shfl_sync(0xffffffffu, cur_c, 0);
+      if (__all_sync(0xffffffffu, cur_c == c0) && c0 >= 0) {
+        const uint32_t r = __reduce_add_sync(0xffffffffu, rc_c);
+        if ((tid & 31) == 0) atomicAdd(&sh.cnt_c[buf][c0], r);
+      } else if (cur_c >= 0) {
+        atomicAdd(&sh.cnt_c[buf][cur_c], rc_c);
+      }
+    }
+    if (use_mass) {
+      const int c0 = __shfl_sync(0xffffffffu, cur_t, 0);
+      if (__all_sync(0xffffffffu, cur_t == c0) && c0 >= 0) {
+        const uint32_t r = __reduce_add_sync(0xffffffffu, rc_t);
+        for (int o = 16; o > 0; o >>= 1) rm_t += __shfl_xor_sync(0xffffffffu, rm_t, o);
         if ((tid & 31) == 0) {
-          atomicAdd(&sh.cnt[buf][cur0], rc);
-          if (by_mass) atomicAdd(&sh.mass[buf][cur0], rm);
+          atomicAdd(&sh.cnt_t[buf][c0], r);
+          atomicAdd(&sh.mass_t[buf][c0], rm_t);
         }
-      } else if (cur >= 0) {
-        atomicAdd(&sh.cnt[buf][cur], rc);
-        if (by_mass) atomicAdd(&sh.mass[buf][cur], rm);
+      } else if (cur_t >= 0) {
+        atomicAdd(&sh.cnt_t[buf][cur_t], rc_t);
+        atomicAdd(&sh.mass_t[buf][cur_t], rm_t);
       }
-      cl.sync();
-      if (tid < 256) {
-        uint32_t c = 0;
-        double m = 0.0;
-        for (int r = 0; r < C; ++r) {
-          c += cl.map_shared_rank(&sh.cnt[buf][0], r)[tid];
-          if (by_mass) m += cl.map_shared_rank(&sh.mass[buf][0], r)[tid];
-        }
-        sh.tot_c[tid] = c;
-        sh.tot_m[tid] = m;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        int bs = -1, last_nonempty = -1;
-        uint32_t ca = cabove;
-        double ma = mabove;
-        for (int b = 255; b >= 0; --b) {
-          const uint32_t c = sh.tot_c[b];
-          if (c == 0) continue;
-          last_nonempty = b;
-          if (by_mass ? (ma + sh.tot_m[b] >= target) : (ca + c >= (uint32_t)k_target)) {
-            bs = b;
-            break;
-          }
-          ca += c;
-          ma += sh.tot_m[b];
-        }
-        if (bs < 0) {  // rounding left the total just short: take the last group
-          bs = last_nonempty;
-          ca -= sh.tot_c[bs];
-          ma -= sh.tot_m[bs];
-        }
-        sh.bstar = bs;
-        sh.cabove = ca;
-        sh.mabove = ma;
-        sh.eqcnt = sh.tot_c[bs];
-      }
-      __syncthreads();
-      prefix |= static_cast<uint32_t>(sh.bstar) << shift;
-      pmask |= 255u << shift;
-      cabove = sh.cabove;
-      mabove = sh.mabove;
-      eqcnt = sh.eqcnt;
-      buf ^= 1;
     }
-    if (by_mass) {
-      const double pstar = pmass(prefix, kmax, smax);
-      const double need = target - mabove;
-      double mm = pstar > 0.0 ? ceil(need / pstar) : static_cast<double>(eqcnt);
-      mm = fmin(fmax(mm, 1.0), static_cast<double>(eqcnt));
-      const int k = static_cast<int>(cabove) + static_cast<int>(mm);
-      if (k > a.k_or_cap) {  // cap binds: keep the top k_or_cap instead
-        by_mass = false;
-        k_target = a.k_or_cap;
-        continue;
+    cl.sync();
+    if (tid < 256) {  // merge the cluster's histograms (same order in every CTA)
+      uint32_t cc = 0, ct = 0;
+      double mt = 0.0;
+      for (int r = 0; r < C; ++r) {
+        cc += cl.map_shared_rank(&sh.cnt_c[buf][0], r)[tid];
+        if (use_mass) {
+          ct += cl.map_shared_rank(&sh.cnt_t[buf][0], r)[tid];
+          mt += cl.map_shared_rank(&sh.mass_t[buf][0], r)[tid];
+        }
       }
-      k_target = k;
+      sh.tot_cc[tid] = cc;
+      sh.tot_ct[tid] = ct;
+      sh.tot_mt[tid] = mt;
     }
-    break;
+    __syncthreads();
+    if (tid == 0) {  // count path: first bucket from the top reaching k_count
+      int bs = -1;
+      uint32_t ca = cab_c;
+      for (int b = 255; b >= 0; --b) {
+        const uint32_t c = sh.tot_cc[b];
+        if (c == 0) continue;
+        if (ca + c >= (uint32_t)k_count) {
+          bs = b;
+          break;
+        }
+        ca += c;
+      }
+      sh.bstar_c = bs;
+      sh.cabove_c = ca;
+    }
+    if (use_mass && tid == 32) {  // mass path: first bucket reaching tau * Z
+      double tg = target;
+      if (pass == 0) {
+        double z = 0.0;
+        for (int b = 255; b >= 0; --b) z += sh.tot_mt[b];
+        tg = a.tau * z;
+        sh.target = tg;
+      }
+      int bs = -1, last_nonempty = -1;
+      uint32_t ca = cab_t;
+      double ma = mab_t;
+      for (int b = 255; b >= 0; --b) {
+        const uint32_t c = sh.tot_ct[b];
+        if (c == 0) continue;
+        last_nonempty = b;
+        if (ma + sh.tot_mt[b] >= tg) {
+          bs = b;
+          break;
+        }
+        ca += c;
+        ma += sh.tot_mt[b];
+      }
+      if (bs < 0) {  // rounding left the total just short: take the last group
+        bs = last_nonempty;
+        ca -= sh.tot_ct[bs];
+        ma -= sh.tot_mt[bs];
+      }
+      sh.bstar_t = bs;
+      sh.cabove_t = ca;
+      sh.mabove_t = ma;
+      sh.eqcnt_t = sh.tot_ct[bs];
+    }
+    __syncthreads();
+    pf_c |= static_cast<uint32_t>(sh.bstar_c) << shift;
+    pm_c |= 255u << shift;
+    cab_c = sh.cabove_c;
+    if (use_mass) {
+      if (pass == 0) target = sh.target;
+      pf_t |= static_cast<uint32_t>(sh.bstar_t) << shift;
+      pm_t |= 255u << shift;
+      cab_t = sh.cabove_t;
+      mab_t = sh.mabove_t;
+      eq_t = sh.eqcnt_t;
+    }
+    buf ^= 1;
   }
-  const uint32_t T = prefix;
+  uint32_t T = pf_c;
+  uint32_t cabove = cab_c;
+  int k_target = k_count;
+  if (use_mass) {
+    // within the final group of equal keys every entry has the same mass
+    const double pstar = pmass(pf_t, kmax, smax);
+    double mm = pstar > 0.0 ? ceil((target - mab_t) / pstar) : static_cast<double>(eq_t);
+    mm = fmin(fmax(mm, 1.0), static_cast<double>(eq_t));
+    const int k_thr = static_cast<int>(cab_t) + static_cast<int>(mm);
+    if (k_thr <= a.k_or_cap) {
+      T = pf_t;
+      cabove = cab_t;
+      k_target = k_thr;
+    }
+  }
   const int m_eq = k_target - static_cast<int>(cabove);  // equal keys to keep (smallest indices)
 
   // ---- ascending compaction across the cluster
@@ -333,6 +379,10 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
                           cudaStream_t stream) {
   int C = (N + 4095) / 4096;
   C = C < 1 ? 1 : (C > kSelMaxCluster ? kSelMaxCluster : C);
+  // Few heads leave most SMs idle: split long rows over 16-CTA clusters.
+  const bool wide = C == kSelMaxCluster && H * kSelMaxCluster * 2 <= device_sm_count() &&
+                    N >= 16 * 4096;
+  if (wide) C = 16;
   const int chunk = (N + C - 1) / C;
   const bool cache = chunk <= kSelCacheKeys;
   SelArgs a{scores, N, ld, mode, k_or_cap, tau, idx, ld_idx, count, status, chunk};
@@ -353,8 +403,18 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
     e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)cfg.dynamicSmemBytes);
     if (e != cudaSuccess) return e;
+    if (wide) {
+      e = cudaFuncSetAttribute(select_kernel<true>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
     e = cudaLaunchKernelEx(&cfg, select_kernel<true>, a);
   } else {
+    if (wide) {
+      e = cudaFuncSetAttribute(select_kernel<false>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
     e = cudaLaunchKernelEx(&cfg, select_kernel<false>, a);
   }
   if (e != cudaSuccess) return e;
