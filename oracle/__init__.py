@@ -22,6 +22,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 TOPK = 0
 THRESHOLD = 1
+MAXFRAC = 2
 
 
 def build(force: bool = False) -> str:

@@ -36,6 +36,7 @@
 
 #define OR_TOPK 0
 #define OR_THRESHOLD 1
+#define OR_MAXFRAC 2
 
 static double load_elem(const void* base, int dtype, int64_t off) {
   if (dtype == OR_BF16) {
@@ -57,6 +58,15 @@ static double load_elem(const void* base, int dtype, int64_t off) {
  * s_max and p_r = 0 for NaN; Z = sum of p_r in the sorted order; k is the
  * smallest k >= 1 whose prefix sum reaches tau*Z (>=); tau == 1 keeps every
  * entry with p_r > 0; Z == 0 gives k = 1; then k = min(k, cap).
+ * MAXFRAC (FlashPrefill summary page, section 2B, "max-based dynamic
+ * thresholding": an entry survives when its score is at least alpha times
+ * the largest score; no sort, no cumulative sum).  The score of an entry is
+ * its softmax mass, so the rule is p_r / Z >= alpha * p_max / Z, i.e.
+ * exp(s_r - s_max) >= alpha, taken in the log domain as
+ *     keep r  iff  s_r == s_max  or  (double)s_r - (double)s_max >= log(alpha)
+ * with `tau` carrying alpha in (0, 1]; NaN is never kept; when every score
+ * is NaN, k = 1; then k = min(k, cap).  The kept entries are a prefix of the
+ * order above, so the output is that prefix.
  * Output: the k indices in ascending order, padded with -1 up to k_or_cap.
  * `margin` receives min(|prefix(k-1) - tau Z|, |prefix(k) - tau Z|) / Z for
  * the threshold decision (+inf for TOPK, and +inf when the uncapped k exceeds
@@ -88,7 +98,8 @@ static int cmp_i32(const void* a, const void* b) {
 int or_select(const float* s, int N, int mode, int k_or_cap, double tau, int32_t* idx,
               int32_t* count, double* margin) {
   if (N < 1 || k_or_cap < 1 || k_or_cap > N) return -1;
-  if (mode == OR_THRESHOLD && !(tau > 0.0 && tau <= 1.0)) return -1;
+  if (mode != OR_TOPK && mode != OR_THRESHOLD && mode != OR_MAXFRAC) return -1;
+  if (mode != OR_TOPK && !(tau > 0.0 && tau <= 1.0)) return -1;
   or_pair* v = (or_pair*)malloc(sizeof(or_pair) * (size_t)N);
   for (int r = 0; r < N; ++r) {
     v[r].s = s[r];
@@ -99,6 +110,16 @@ int or_select(const float* s, int N, int mode, int k_or_cap, double tau, int32_t
   *margin = INFINITY;
   if (mode == OR_TOPK) {
     k = k_or_cap;
+  } else if (mode == OR_MAXFRAC) {
+    const double smax = (double)v[0].s, lna = log(tau);
+    k = 0;
+    for (int r = 0; r < N; ++r) {
+      const double x = (double)v[r].s;
+      if (isnan(x)) continue;
+      if (x == smax || x - smax >= lna) ++k;
+    }
+    if (k < 1) k = 1;
+    if (k > k_or_cap) k = k_or_cap;
   } else {
     double smax = (double)v[0].s;
     double* p = (double*)malloc(sizeof(double) * (size_t)N);
