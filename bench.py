@@ -237,7 +237,7 @@ def run_ours(args, w):
     N, Hq, d = Q.shape
     Hkv = K.shape[1]
     H_sel = w.H_sel
-    mode = vs.VS_SELECT_TOPK if w.select_mode == "topk" else vs.VS_SELECT_THRESHOLD
+    mode = w.select_mode_id
     if w.indexer:
         W1d, W2d = torch.from_numpy(W1).to(dev), torch.from_numpy(W2).to(dev)
         LV = torch.empty((Hkv, N), dtype=torch.float32, device=dev)
@@ -254,9 +254,12 @@ def run_ours(args, w):
     ws_sel2 = vs.workspace(vs.vs_select_workspace_size(H_sel, N), dev)
     ws_att = vs.workspace(vs.vs_attn_workspace_size_ld(N, Hq, H_sel, d, w.k_v), dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    launches_per_step = 4 + (1 if w.indexer else 0)
+    # select x2, plan, pack (when each index set's heads lie in one KV group), attention,
+    # plus the indexer; the status-word resets are driver memsets, not counted
+    packs = (Hq // Hkv) % (Hq // H_sel) == 0
+    launches_per_step = 4 + (1 if packs else 0) + (1 if w.indexer else 0)
 
-    ev = {k: [] for k in ("step0", "att0", "att1", "step1")}
+    ev = {k: [] for k in ("step0", "idx1", "att0", "att1", "step1")}
 
     def step(record):
         if record:
@@ -265,6 +268,10 @@ def run_ours(args, w):
             ev["step0"].append(e)
         if w.indexer:
             vs.vs_index_scores(K, V, W1d, W2d, LV, LS)
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev["idx1"].append(e)
         vs.vs_select(LV, mode, w.k_v, w.tau_v, vi, vc, ws_sel)
         vs.vs_select(LS, mode, w.k_s, w.tau_s, si, sc, ws_sel2)
         if record:
@@ -306,10 +313,12 @@ def run_ours(args, w):
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in zip(ev["step0"], ev["step1"])]
     att_ms = [a.elapsed_time(b) for a, b in zip(ev["att0"], ev["att1"])]
-    sel_ms = [a.elapsed_time(b) for a, b in zip(ev["step0"], ev["att0"])]
+    sel_ms = [a.elapsed_time(b) for a, b in zip(ev["idx1"], ev["att0"])]
+    idx_ms = [a.elapsed_time(b) for a, b in zip(ev["step0"], ev["idx1"])]
     ms_step = float(np.mean(step_ms))
     ms_att = float(np.mean(att_ms))
     ms_sel = float(np.mean(sel_ms))
+    ms_idx = float(np.mean(idx_ms))
     ms_step, ms_att = max_over_ranks([ms_step, ms_att], dev)
     value = whole_job_value(world, flops, ms_step)
 
@@ -385,8 +394,10 @@ def run_ours(args, w):
                    "tau_s": w.tau_s, "indexer": w.indexer, "parallelism": f"replicas x{world}",
                    "l2": "inputs exceed L2 (Q/K/V/O resident in HBM) and a 256 MiB buffer is "
                          "written between timed steps, outside the timed windows"},
-        "ms_per_layer": round(ms_step, 3), "ms_select": round(ms_sel, 3),
-        "ms_attention": round(ms_att, 3),
+        "ms_per_layer": round(ms_step, 3), "ms_indexer": round(ms_idx, 3) if w.indexer else None,
+        "ms_select": round(ms_sel, 3), "ms_attention": round(ms_att, 3),
+        "kernels": kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, algo_bytes, ms_att,
+                                    ms_sel, ms_idx, vih.shape[1], sih.shape[1]),
         "selected_pairs": int(P_total), "density_vs_causal": round(P_total / (Hq * N * (N + 1) / 2), 5),
         "dense_ms": None if dense_ms is None else round(dense_ms, 3),
         "dense_tflops": None if dense_ms is None else round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
@@ -410,6 +421,34 @@ def run_ours(args, w):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, att_bytes, ms_att, ms_sel, ms_idx,
+                     ld_v, ld_s):
+    """Per hot-path kernel: achieved vs the roofline that bounds it.
+    attention (+plan, +pack): tensor-bound, 4 d P flops; select x2: HBM-bound,
+    4 B per score read + 4 B per index slot written; indexer: fp32 CUDA-core
+    FMA-bound, 2 (2d hidden + 2 hidden) flops per (token, KV head), peak =
+    148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz."""
+    out = {}
+    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    t_att = flops / (peak_t * 1e12)
+    out["attention"] = {"ms": round(ms_att, 3), "bound": "tensor",
+                        "achieved_tflops": round(flops / (ms_att * 1e-3) / 1e12, 2),
+                        "frac": round(max(t_att, att_bytes / (peaks["hbm_gbs"] * 1e9)) / (ms_att * 1e-3), 4)}
+    sel_bytes = 4.0 * H_sel * N * 2 + 4.0 * H_sel * (ld_v + ld_s)
+    out["select_x2"] = {"ms": round(ms_sel, 3), "bound": "hbm",
+                        "achieved_gbs": round(sel_bytes / (ms_sel * 1e-3) / 1e9, 1),
+                        "frac": round(sel_bytes / (peaks["hbm_gbs"] * 1e9) / (ms_sel * 1e-3), 5)}
+    if w.indexer:
+        hidden = w.hidden
+        iflops = 2.0 * N * Hkv * (2 * d * hidden + 2 * hidden)
+        alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6
+        out["indexer"] = {"ms": round(ms_idx, 3), "bound": "alu",
+                          "achieved_tflops": round(iflops / (ms_idx * 1e-3) / 1e12, 2),
+                          "peak_tflops": round(alu_peak / 1e12, 1),
+                          "frac": round(iflops / alu_peak / (ms_idx * 1e-3), 4)}
+    return out
 
 
 def structural_touched(N, vi, vc, si, sc, Hq):
@@ -484,7 +523,7 @@ def run_reference(args, w):
         return
     import oracle
     Qb, Kb, Vb = w.qkv()
-    mode = oracle.TOPK if w.select_mode == "topk" else oracle.THRESHOLD
+    mode = w.select_mode_id
     if w.indexer:
         W1, W2 = w.indexer_weights()
         toks = np.arange(w.N)

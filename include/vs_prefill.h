@@ -59,7 +59,7 @@ typedef enum {
   VS_ERR_DEVICE_BOUNDS = 6   /* returned by vs_read_device_status */
 } vs_status;
 
-typedef enum { VS_SELECT_TOPK = 0, VS_SELECT_THRESHOLD = 1 } vs_select_mode;
+typedef enum { VS_SELECT_TOPK = 0, VS_SELECT_THRESHOLD = 1, VS_SELECT_MAXFRAC = 2 } vs_select_mode;
 
 typedef enum { VS_BF16 = 0, VS_FP32 = 1 } vs_dtype;
 
@@ -109,13 +109,22 @@ vs_status vs_index_scores(const void* K, const void* V, vs_dtype dtype, int N, i
  *            tau (0 < tau <= 1): p_r = exp(s_r - s_max) in fp64, k is the
  *            smallest k >= 1 with sum_{r<k} p_r >= tau * sum_r p_r; tau = 1
  *            keeps every entry with p_r > 0; then k = min(k, k_or_cap).
+ *   MAXFRAC  FlashPrefill's max-based dynamic threshold (FlashPrefill summary
+ *            page, section 2B: discard every candidate scoring below alpha
+ *            times the best one; no sort, no cumulative sum).  `tau` carries
+ *            alpha (0 < alpha <= 1); with the mass reading the rule is
+ *            p_r >= alpha, decided in fp64 as
+ *              s_r == s_max  or  (double)s_r - (double)s_max >= log(alpha)
+ *            (log taken on the host); NaN is never kept, an all-NaN row
+ *            keeps one entry; then k = min(k, k_or_cap) in the order above.
  *   idx      int32 [H][ld_idx] (device): for each head the kept indices in
  *            ascending order, then -1 up to k_or_cap (entries past k_or_cap
  *            untouched).  ld_idx >= k_or_cap.
  *   count    int32 [H] (device): kept entries per head.
  *   ws       device workspace of at least vs_select_workspace_size(H, N)
  *            bytes, 256-byte aligned (holds the device status word).
- * Requires 1 <= k_or_cap <= N <= 2^20.
+ * Requires 1 <= k_or_cap <= N <= 2^20; tau in (0, 1] for THRESHOLD and
+ * MAXFRAC (else VS_ERR_INVALID_ARG).
  */
 size_t vs_select_workspace_size(int H, int N);
 vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_select_mode mode,

@@ -30,6 +30,7 @@ VS_ERR_DEVICE_BOUNDS = 6
 
 VS_SELECT_TOPK = 0
 VS_SELECT_THRESHOLD = 1
+VS_SELECT_MAXFRAC = 2
 VS_BF16 = 0
 VS_FP32 = 1
 

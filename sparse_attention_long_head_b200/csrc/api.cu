@@ -117,13 +117,15 @@ vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_sel
   if (!scores || !idx || !count) return VS_ERR_INVALID_ARG;
   if (H < 1 || H > 65535 || N < 1 || ld_scores < N) return VS_ERR_INVALID_ARG;
   if (N > (1 << 20)) return VS_ERR_UNSUPPORTED;
-  if (mode != VS_SELECT_TOPK && mode != VS_SELECT_THRESHOLD) return VS_ERR_INVALID_ARG;
+  if (mode != VS_SELECT_TOPK && mode != VS_SELECT_THRESHOLD && mode != VS_SELECT_MAXFRAC)
+    return VS_ERR_INVALID_ARG;
   if (k_or_cap < 1 || k_or_cap > N || ld_idx < k_or_cap) return VS_ERR_INVALID_ARG;
-  if (mode == VS_SELECT_THRESHOLD && !(tau > 0.0 && tau <= 1.0)) return VS_ERR_INVALID_ARG;
+  if (mode != VS_SELECT_TOPK && !(tau > 0.0 && tau <= 1.0)) return VS_ERR_INVALID_ARG;
+  const double ln_alpha = mode == VS_SELECT_MAXFRAC ? std::log(tau) : 0.0;
   if (!ws || ws_bytes < vs_select_workspace_size(H, N) || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
   int* status = static_cast<int*>(ws);
   if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
-  if (launch_select(scores, H, N, ld_scores, mode, k_or_cap, tau, idx, ld_idx, count, status,
+  if (launch_select(scores, H, N, ld_scores, mode, k_or_cap, tau, ln_alpha, idx, ld_idx, count, status,
                     stream) != cudaSuccess)
     return VS_ERR_CUDA;
   return VS_OK;

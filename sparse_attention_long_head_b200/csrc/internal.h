@@ -149,7 +149,7 @@ cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_attn_tc(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_attn_fp32(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,
-                          double tau, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
+                          double tau, double ln_alpha, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
                           cudaStream_t stream);
 cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, int Hkv, int d,
                                 int64_t stride_tok, int64_t stride_head, const float* W1,

@@ -22,6 +22,10 @@
 //     histogram); inside the final group of equal keys the count follows from
 //     their common mass.  The top-cap boundary is searched in the same passes,
 //     so a capped head needs no second search.
+//   * FlashPrefill's max-based rule (summary page, section 2B: keep what
+//     scores at least alpha times the maximum, no sort and no cumulative sum)
+//     is one counting pass after the maximum; the kept entries are all keys
+//     at or above a boundary, so unless the cap binds no search runs at all.
 //   * A last pass writes the kept indices in ascending order (index-ordered
 //     compaction across the cluster), then pads with -1.
 #include <cooperative_groups.h>
@@ -55,6 +59,7 @@ struct SelArgs {
   int mode;
   int k_or_cap;
   double tau;
+  double ln_alpha;  // max-based rule: log(alpha), computed once on the host
   int32_t* idx;
   int64_t ld_idx;
   int32_t* count;
@@ -70,6 +75,7 @@ struct SelShared {
   double tot_mt[256];
   uint32_t kmax;
   uint32_t npos;
+  uint32_t kmin_kept;
   uint32_t gt, eq;
   int bstar_c, bstar_t;
   uint32_t cabove_c, cabove_t, eqcnt_t;
@@ -153,7 +159,43 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   // count path's top-cap result (k = min(k_threshold, cap)).
   int k_count = a.k_or_cap;
   bool use_mass = false;
-  if (a.mode == VS_SELECT_THRESHOLD) {
+  bool search = true;            // false: the kept set is every key >= kmin_kept
+  uint32_t kmin_kept = 0xFFFFFFFFu;
+  if (a.mode == VS_SELECT_MAXFRAC) {
+    // keep r iff key_r == kmax or (double)s_r - s_max >= log(alpha); NaN
+    // (key 0) never.  The test is monotone in the key, so the kept entries
+    // are the keys >= the smallest kept key.
+    uint32_t c = 0, kmin = 0xFFFFFFFFu;
+    if (kmax != 0u) {
+      for (int e = tid; e < n; e += nt) {
+        const uint32_t k = key_at(e);
+        if (k != 0u && (k == kmax || static_cast<double>(fkey_inv(k)) - smax >= a.ln_alpha)) {
+          ++c;
+          kmin = min(kmin, k);
+        }
+      }
+    }
+    c = static_cast<uint32_t>(block_reduce<int>(static_cast<int>(c), sh.wred_i,
+                                                [](int x, int y) { return x + y; }));
+    kmin = block_reduce<int>(static_cast<int>(kmin ^ 0x80000000u), sh.wred_i,
+                             [](int x, int y) { return x < y ? x : y; }) ^ 0x80000000u;
+    if (tid == 0) {
+      sh.npos = c;
+      sh.kmin_kept = kmin;
+    }
+    cl.sync();
+    int tot = 0;
+    for (int r = 0; r < C; ++r) {
+      tot += static_cast<int>(*cl.map_shared_rank(&sh.npos, r));
+      kmin_kept = min(kmin_kept, *cl.map_shared_rank(&sh.kmin_kept, r));
+    }
+    if (kmax == 0u) {  // every score is NaN: keep one entry
+      k_count = 1;
+    } else if (tot <= a.k_or_cap) {
+      k_count = tot;
+      search = false;
+    }
+  } else if (a.mode == VS_SELECT_THRESHOLD) {
     if (kmax == 0u) {  // every score is NaN: keep one entry
       k_count = 1;
     } else if (a.tau >= 1.0) {  // keep every entry with p > 0
@@ -175,7 +217,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   uint32_t pf_t = 0, pm_t = 0, cab_t = 0, eq_t = 0;  // mass path
   double mab_t = 0.0, target = 0.0;
   int buf = 0;
-  for (int pass = 0; pass < 4; ++pass) {
+  for (int pass = 0; pass < (search ? 4 : 0); ++pass) {
     const int shift = 24 - 8 * pass;
     if (tid < 256) {
       sh.cnt_c[buf][tid] = 0;
@@ -319,6 +361,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   uint32_t T = pf_c;
   uint32_t cabove = cab_c;
   int k_target = k_count;
+  if (!search) {  // every key > kmin_kept - 1 is kept; no equal-key group to trim
+    T = kmin_kept - 1u;
+    cabove = static_cast<uint32_t>(k_count);
+  }
   if (use_mass) {
     // within the final group of equal keys every entry has the same mass
     const double pstar = pmass(pf_t, kmax, smax);
@@ -375,7 +421,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
 }
 
 cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,
-                          double tau, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
+                          double tau, double ln_alpha, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
                           cudaStream_t stream) {
   int C = (N + 4095) / 4096;
   C = C < 1 ? 1 : (C > kSelMaxCluster ? kSelMaxCluster : C);
@@ -385,7 +431,7 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
   if (wide) C = 16;
   const int chunk = (N + C - 1) / C;
   const bool cache = chunk <= kSelCacheKeys;
-  SelArgs a{scores, N, ld, mode, k_or_cap, tau, idx, ld_idx, count, status, chunk};
+  SelArgs a{scores, N, ld, mode, k_or_cap, tau, ln_alpha, idx, ld_idx, count, status, chunk};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, H, 1);
   cfg.blockDim = dim3(kSelThreads, 1, 1);

@@ -83,6 +83,10 @@ def test_select_host_validation():
     assert call(mode=1, tau=0.0) == vs.VS_ERR_INVALID_ARG
     assert call(mode=1, tau=1.5) == vs.VS_ERR_INVALID_ARG
     assert call(mode=1, tau=float("nan")) == vs.VS_ERR_INVALID_ARG
+    assert call(mode=2, tau=0.0) == vs.VS_ERR_INVALID_ARG
+    assert call(mode=2, tau=1.0000001) == vs.VS_ERR_INVALID_ARG
+    assert call(mode=2, tau=float("nan")) == vs.VS_ERR_INVALID_ARG
+    assert call(mode=3) == vs.VS_ERR_INVALID_ARG
     assert call(ws=None) == vs.VS_ERR_WORKSPACE
     assert call(wsb=16) == vs.VS_ERR_WORKSPACE
     assert call(ws=_fake(0x20010)) == vs.VS_ERR_WORKSPACE  # misaligned

@@ -10,21 +10,22 @@ from vs_workloads import WORKLOADS
 
 pytestmark = pytest.mark.gpu
 
-TOPK, THR = vs.VS_SELECT_TOPK, vs.VS_SELECT_THRESHOLD
+TOPK, THR, MAXF = vs.VS_SELECT_TOPK, vs.VS_SELECT_THRESHOLD, vs.VS_SELECT_MAXFRAC
 
 
 @pytest.mark.parametrize("name", ["tiny_1k", "llama_8k", "llama_32k", "llama_128k", "llama_128k_S"])
 def test_workload_scores(name, cuda_device):
     w = WORKLOADS[name]
     lv, ls = w.all_scores()
-    mode = TOPK if w.select_mode == "topk" else THR
+    mode = w.select_mode_id
     ties = check_select(lv, mode, w.k_v, w.tau_v)
     ties += check_select(ls, mode, w.k_s, w.tau_s)
     assert ties == [], f"tie zones at heads {ties}"
 
 
 @pytest.mark.parametrize("N", [1, 2, 100, 4095, 4096, 4097, 33000, 131071])
-@pytest.mark.parametrize("mode,tau", [(TOPK, 1.0), (THR, 0.5), (THR, 0.95), (THR, 1.0)])
+@pytest.mark.parametrize("mode,tau", [(TOPK, 1.0), (THR, 0.5), (THR, 0.95), (THR, 1.0),
+                                      (MAXF, 0.5), (MAXF, 1e-3), (MAXF, 1.0)])
 def test_sizes_and_modes(N, mode, tau, cuda_device):
     rng = np.random.default_rng(N)
     s = (rng.standard_normal((3, N)) * 2).astype(np.float32)
@@ -51,6 +52,12 @@ def test_ties_nan_inf_signed_zero(cuda_device):
     check_select(allnan, TOPK, 10)
     allneg = np.full((1, 5000), -np.inf, np.float32)
     check_select(allneg, THR, 5000, 0.5)
+    for alpha in (1.0, 0.2, 1e-30):
+        check_select(s, MAXF, N, alpha)
+        check_select(s, MAXF, 100, alpha)
+    check_select(allnan, MAXF, 10, 0.5)
+    check_select(allneg, MAXF, 5000, 0.5)
+    check_select(allneg, MAXF, 17, 0.5)
 
 
 def test_all_equal_closed_form(cuda_device):
@@ -75,3 +82,41 @@ def test_large_n_without_shared_cache(cuda_device):
     s = rng.standard_normal((2, N)).astype(np.float32)
     check_select(s, TOPK, 12345)
     check_select(s, THR, N, 0.95)
+
+
+@pytest.mark.parametrize("name", ["llama_8k", "llama_128k"])
+@pytest.mark.parametrize("alpha", [0.3, 0.01])
+def test_maxfrac_on_workload_scores(name, alpha, cuda_device):
+    # FlashPrefill's max-based rule on the workloads' score vectors, with the
+    # workload's budgets as caps (binding for some heads, not for others)
+    w = WORKLOADS[name]
+    lv, ls = w.all_scores()
+    assert check_select(lv, MAXF, w.k_v, alpha) == []
+    assert check_select(ls, MAXF, w.k_s, alpha) == []
+    assert check_select(lv, MAXF, w.N, alpha) == []
+
+
+def test_maxfrac_exact_boundary_is_kept(cuda_device):
+    import math
+    rows = []
+    for q in range(1, 200):
+        d = -q / 8.0
+        if math.log(math.exp(d)) == d:
+            rows.append((d, math.exp(d)))
+    assert len(rows) > 20
+    for d, alpha in rows[:8]:
+        s = np.array([[0.0, d, d - 0.125] + [-1e3] * 5000], np.float32)
+        check_select(s, MAXF, 5003, alpha)
+        check_select(s, MAXF, 1, alpha)
+
+
+def test_maxfrac_near_uniform_long_rows(cuda_device):
+    # the indexer workload's shape: 8 heads x 262144 near-uniform logits
+    # (std 0.06); alpha decides between a binding cap and a short list
+    rng = np.random.default_rng(7)
+    s = (0.06 * rng.standard_normal((8, 262144))).astype(np.float32)
+    check_select(s, MAXF, 16384, 0.5)   # ~all entries pass: the cap binds
+    check_select(s, MAXF, 16384, 0.9)  # a few hundred entries pass: no search
+    big = rng.standard_normal((2, 300000)).astype(np.float32)  # beyond the shared cache
+    check_select(big, MAXF, 300000, 0.05)
+    check_select(big, MAXF, 1000, 0.05)

@@ -199,7 +199,7 @@ class Workload:
     d: int
     rope_base: float
     seed: int
-    select_mode: str            # "topk" | "threshold"
+    select_mode: str            # "topk" | "threshold" | "maxfrac"
     k_v: int                    # top-k budget or cap
     k_s: int
     tau_v: float = 1.0
@@ -209,6 +209,11 @@ class Workload:
     hidden: int = 256
     description: str = ""
     extra: dict = field(default_factory=dict)
+
+    @property
+    def select_mode_id(self) -> int:
+        """The rule's number in the C ABI and the oracle (0 top-k, 1 threshold, 2 max-based)."""
+        return {"topk": 0, "threshold": 1, "maxfrac": 2}[self.select_mode]
 
     @property
     def H_sel(self) -> int:
@@ -260,6 +265,11 @@ WORKLOADS = {
                              8192, tau_v=0.95, tau_s=0.95, heads="local_global_S",
                              description="variant of llama_128k whose global heads draw "
                                          "structured (local) slash scores"),
+    "llama_128k_maxfrac": Workload("llama_128k_maxfrac", 131072, 32, 8, 128, 500000.0, 14,
+                                   "maxfrac", 8192, 8192, tau_v=1e-3, tau_s=1e-3,
+                                   heads="local_global",
+                                   description="llama_128k's inputs with FlashPrefill's max-based "
+                                               "rule: keep mass >= 1e-3 x the largest, cap 8192"),
     "llama_256k_indexer": Workload("llama_256k_indexer", 262144, 32, 8, 128, 500000.0, 15,
                                    "threshold", 16384, 16384, tau_v=0.95, tau_s=0.95, indexer=True,
                                    description="32q/8kv, d=128, N=262144, scores from the "
