@@ -482,8 +482,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + 2 * C::kQBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kData);
-  enum { B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 6, B_OEMPTY = 8,
-         B_DRAIN = 10, B_FULL = 11, B_EMPTY = 11 + S, B_END = 11 + 2 * S };
+  // K/V tiles stream through an S-slot ring in the order K(0), V(0), K(1),
+  // V(1), ... of each unit.  They are grouped into stages that complete on one
+  // barrier each: [K(0)], [V(0), K(1)], ..., [V(n-2), K(n-1)], [V(n-1)], so
+  // that one wait of the MMA issuer covers both tiles a step needs.  Every
+  // stage holds at least one tile, so at most S stages are in flight and S
+  // stage barriers suffice.
+  enum { B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 6, B_DRAIN = 8,
+         B_STAGE = 9, B_EMPTY = 9 + S, B_END = 9 + 2 * S };
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + B_END);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -496,11 +502,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(B_SFULL + s), 1);
       mbar_init(bar(B_PFULL + s), 128);
       mbar_init(bar(B_OFULL + s), 1);
-      mbar_init(bar(B_OEMPTY + s), 128);
     }
     mbar_init(bar(B_DRAIN), 1);
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_STAGE + s), 1);
       mbar_init(bar(B_EMPTY + s), 1);
     }
     *abort_flag = 0;
@@ -638,8 +643,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (i < P.N && P.lse)
         P.lse[(int64_t)ui.h * P.N + i] =
             l > 0.f ? (m_use + log2f(l)) * 0.6931471805599453f : -INFINITY;
-      tc_fence_before();
-      mbar_arrive(bar(B_OEMPTY + sub));
       ++ucount;
     }
   } else if (warp == kWarpMMA) {
@@ -648,7 +651,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), kv_addr = smem_u32(sKV);
-      uint32_t seq = 0, ucount = 0, pcnt[2] = {0, 0};
+      uint32_t seq = 0, stg = 0, ucount = 0, pcnt[2] = {0, 0};
       bool ok = true;
       // Descriptors of the tile bases; per-MMA k offsets are compile-time
       // constants added to the 14-bit start-address field (addresses < 256 KB,
@@ -678,8 +681,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ui.n == 0) continue;
         if (!mbar_wait(bar(B_QFULL), ucount & 1, wc)) { ok = false; break; }
         uint32_t kslot = seq % S;
-        if (!mbar_wait(bar(B_FULL + kslot), (seq / S) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait(bar(B_STAGE + stg % S), (stg / S) & 1, wc)) { ok = false; break; }  // [K(0)]
         ++seq;
+        ++stg;
         tc_fence_after();
         issue_s(0, kslot);
         mma_commit(bar(B_SFULL + 0));
@@ -687,20 +691,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mma_commit(bar(B_SFULL + 1));
         mma_commit(bar(B_EMPTY + kslot));
         for (int k = 0; k < ui.n && ok; ++k) {
+          // one wait for V(k) and K(k+1): stage [V(k), K(k+1)] (or [V(n-1)])
+          if (!mbar_wait(bar(B_STAGE + stg % S), (stg / S) & 1, wc)) { ok = false; break; }
+          ++stg;
           const uint32_t vslot = seq % S;
-          if (!mbar_wait(bar(B_FULL + vslot), (seq / S) & 1, wc)) { ok = false; break; }
           ++seq;
-          if (k + 1 < ui.n) {  // next K tile, waited for off the critical path
+          if (k + 1 < ui.n) {
             kslot = seq % S;
-            if (!mbar_wait(bar(B_FULL + kslot), (seq / S) & 1, wc)) { ok = false; break; }
             ++seq;
           }
           for (int sub = 0; sub < 2; ++sub) {
+            // P(k) of this sub-tile; at k = 0 this also means its rows' previous
+            // epilogue has read O (the same threads arrive after it), so PV(0)
+            // may overwrite O
             if (!mbar_wait(bar(B_PFULL + sub), pcnt[sub] & 1, wc)) { ok = false; break; }
             ++pcnt[sub];
-            if (k == 0 && ucount > 0) {
-              if (!mbar_wait(bar(B_OEMPTY + sub), (ucount - 1) & 1, wc)) { ok = false; break; }
-            }
             tc_fence_after();
             issue_pv(sub, vslot, k > 0);
             if (sub == 1) mma_commit(bar(B_EMPTY + vslot));
@@ -723,7 +728,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == kWarpLoad) {
     // ------------------------------------------------------- TMA producer
-    uint32_t seq = 0, ucount = 0;
+    uint32_t seq = 0, stg = 0, ucount = 0;
     bool ok = true;
     const int nsub64 = D / 64;
     for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
@@ -738,16 +743,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         ui.h * D + 64 * h, 256 * ui.p + 128 * s);
       }
       ++ucount;
-      for (int k = 0; k < ui.n && ok; ++k) {
+      // tile t of the unit: K(t/2) for even t, V(t/2) for odd t; a stage
+      // starts at t = 0 and at every odd t, and holds two tiles except the
+      // first and the last
+      const int ntiles = 2 * ui.n;
+      for (int t = 0; t < ntiles && ok; ++t) {
+        const int k = t >> 1, kv = t & 1;
         const Item it = unit_item(P, ui, k);
-        for (int kv = 0; kv < 2; ++kv) {
+        {
           const uint32_t slot = seq % S;
           if (seq >= (uint32_t)S && !mbar_wait(bar(B_EMPTY + slot), ((seq / S) - 1) & 1, wc)) {
             ok = false;
             break;
           }
-          const uint32_t fb = bar(B_FULL + slot);
-          if (lane == 0) mbar_arrive_expect_tx(fb, C::kTileBytes);
+          const uint32_t fb = bar(B_STAGE + stg % S);
+          if (t == 0 || kv == 1) {  // first tile of a stage: arm it for all of its bytes
+            const int nst = (t == 0 || t == ntiles - 1) ? 1 : 2;
+            if (lane == 0) mbar_arrive_expect_tx(fb, nst * C::kTileBytes);
+          }
           __syncwarp();
           const uint32_t dst = smem_u32(sKV + slot * C::kTileBytes);
           if (it.kind == kItemTile) {
@@ -778,14 +791,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                           rr[2], rr[3]);
           }
           ++seq;
+          if (t == 0 || kv == 0 || t == ntiles - 1) ++stg;  // the stage's last tile is issued
         }
       }
     }
     // Drain: let every issued copy land before shared memory is released.
     if (lane == 0) {
-      const uint32_t first = seq > (uint32_t)S ? seq - S : 0;
-      for (uint32_t x = first; x < seq; ++x)
-        mbar_wait_drain(bar(B_FULL + (x % S)), (x / S) & 1, P.wait_limit_ns);
+      const uint32_t first = stg > (uint32_t)S ? stg - S : 0;
+      for (uint32_t x = first; x < stg; ++x)
+        mbar_wait_drain(bar(B_STAGE + (x % S)), (x / S) & 1, P.wait_limit_ns);
       if (ucount > 0) mbar_wait_drain(bar(B_QFULL), (ucount - 1) & 1, P.wait_limit_ns);
     }
   }
