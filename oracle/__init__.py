@@ -54,6 +54,9 @@ def _load():
         lib.or_count_pairs.restype = i64
         lib.or_index_scores.argtypes = [P, P, i32, i32, i32, i32, i64, i64, P, P, i32, P, i32, P, P]
         lib.or_index_scores.restype = None
+        lib.or_aggregate.argtypes = [P, P, i32, i32, i32, i32, i32, i64, i64, dbl, P, i32, i64, i64,
+                                     P, P]
+        lib.or_aggregate.restype = None
         _lib = lib
     return _lib
 
@@ -169,3 +172,29 @@ def index_scores(K, V, W1, W2, toks=None):
     _load().or_index_scores(_ptr(K), _ptr(V), dtype, N, Hkv, d, Hkv * d, d, _ptr(W1), _ptr(W2),
                             W1.shape[0], _ptr(toks), toks.size, _ptr(lv), _ptr(ls))
     return lv, ls
+
+
+def aggregate(Q, K, heads=None, rows=None, scale=0.0):
+    """Ground-truth column / diagonal sums of the full causal softmax weights.
+
+    Q [N, Hq, d], K [N, Hkv, d] as bf16 bits (uint16) or float32.  Returns
+    (A_v, A_s), each float64 [len(heads), N].  `rows` = (lo, hi) restricts the
+    contributing query rows (default all); with hi = N, entries j >= lo of A_v
+    and o >= lo of A_s are exact."""
+    if Q.dtype == np.uint16:
+        dtype = 0
+    elif Q.dtype == np.float32:
+        dtype = 1
+    else:
+        raise TypeError("Q/K must be bf16 bits (uint16) or float32")
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    Q = np.ascontiguousarray(Q)
+    K = np.ascontiguousarray(K)
+    heads = np.arange(Hq, dtype=np.int32) if heads is None else np.ascontiguousarray(heads, np.int32)
+    lo, hi = (0, N) if rows is None else rows
+    Av = np.empty((heads.size, N), np.float64)
+    As = np.empty((heads.size, N), np.float64)
+    _load().or_aggregate(_ptr(Q), _ptr(K), dtype, N, Hq, Hkv, d, Hq * d, Hkv * d, float(scale),
+                         _ptr(heads), heads.size, int(lo), int(hi), _ptr(Av), _ptr(As))
+    return Av, As

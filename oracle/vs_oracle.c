@@ -367,3 +367,54 @@ void or_index_scores(const void* K, const void* V, int dtype, int N, int Hkv, in
     free(hh);
   }
 }
+
+/* ------------------------------------------------- ground-truth aggregation
+ * The distillation target of the VSIndexer ("VSPrefill ..." Technical
+ * Summary, section 2, "Distillation Training": a kernel aggregates the full
+ * attention weights along vertical columns and slash diagonals during the
+ * block-wise computation, without materialising the n x n matrix).  For query
+ * head h with full causal softmax weights p_ij (j <= i):
+ *     A_v[j] = sum_{i >= j} p_ij          (column sums)
+ *     A_s[o] = sum_{i >= o} p_{i, i - o}  (sums along the diagonal at offset o)
+ * so that sum_j A_v[j] = sum_o A_s[o] = N.  Scores s_ij = scale * q_i . k_j in
+ * fp64 (inputs upcast exactly); p_ij = exp(s_ij - m_i) / sum_j exp(s_ij - m_i).
+ * Only rows i in [row_lo, row_hi) contribute (the full result for
+ * [0, N)); A_v[j] for j >= row_lo and A_s[o] for o >= row_lo are then exact
+ * when row_hi = N, since no other row reaches them.  Rows are added in
+ * ascending order; OpenMP runs heads in parallel, never one sum.
+ * Av, As: [nheads][N], zeroed here; heads[] lists the query heads. */
+void or_aggregate(const void* Q, const void* K, int dtype, int N, int Hq, int Hkv, int d,
+                  int64_t q_stride_tok, int64_t kv_stride_tok, double scale, const int* heads,
+                  int nheads, int64_t row_lo, int64_t row_hi, double* Av, double* As) {
+  if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int x = 0; x < nheads; ++x) {
+    const int h = heads[x];
+    const int kvh = h / (Hq / Hkv);
+    double* av = Av + (int64_t)x * N;
+    double* as = As + (int64_t)x * N;
+    for (int64_t j = 0; j < N; ++j) av[j] = as[j] = 0.0;
+    double* q = (double*)malloc(sizeof(double) * (size_t)d);
+    double* s = (double*)malloc(sizeof(double) * (size_t)N);
+    for (int64_t i = row_lo; i < row_hi; ++i) {
+      for (int c = 0; c < d; ++c) q[c] = load_elem(Q, dtype, i * q_stride_tok + (int64_t)h * d + c);
+      double m = -INFINITY;
+      for (int64_t j = 0; j <= i; ++j) {
+        const int64_t off = j * kv_stride_tok + (int64_t)kvh * d;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += q[c] * load_elem(K, dtype, off + c);
+        s[j] = scale * dot;
+        if (s[j] > m) m = s[j];
+      }
+      double z = 0.0;
+      for (int64_t j = 0; j <= i; ++j) z += exp(s[j] - m);
+      for (int64_t j = 0; j <= i; ++j) {
+        const double p = exp(s[j] - m) / z;
+        av[j] += p;
+        as[i - j] += p;
+      }
+    }
+    free(q);
+    free(s);
+  }
+}
