@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--dense-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--agg-steps", type=int, default=2,
+                    help="timed runs of the ground-truth aggregation pass (0: skip)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
 
@@ -341,6 +343,33 @@ def run_ours(args, w):
         dense_ms = float(np.mean(ts))
         del Od
 
+    # ground-truth aggregation (column / diagonal sums of the full attention
+    # weights) on the same inputs, after a dense pass for the row LSE
+    agg = None
+    if args.agg_steps > 0:
+        Od = torch.empty_like(Q)
+        lse_d = torch.empty((Hq, N), dtype=torch.float32, device=dev)
+        vs.vs_dense_attn_fwd(Q, K, V, Od, lse_d, ws_dense)
+        del Od
+        A_v = torch.empty((Hq, N), dtype=torch.float32, device=dev)
+        A_s = torch.empty_like(A_v)
+        vs.vs_attn_aggregate(Q, K, lse_d, A_v, A_s, ws_dense)
+        ts = []
+        for _ in range(args.agg_steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            vs.vs_attn_aggregate(Q, K, lse_d, A_v, A_s, ws_dense)
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        rc, flags = vs.vs_read_device_status(ws_dense)
+        if rc != vs.VS_OK:
+            raise RuntimeError(f"aggregate device status {vs.status_string(rc)} flags {flags}")
+        agg = {"ms": float(np.mean(ts)), "row_sum_err": float((A_v.sum(1) - N).abs().max() / N)}
+        del A_v, A_s, lse_d
+
     # end to end through the public API with host buffers (pinned)
     e2e = None
     if not args.no_e2e:
@@ -397,7 +426,7 @@ def run_ours(args, w):
         "ms_per_layer": round(ms_step, 3), "ms_indexer": round(ms_idx, 3) if w.indexer else None,
         "ms_select": round(ms_sel, 3), "ms_attention": round(ms_att, 3),
         "kernels": kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, algo_bytes, ms_att,
-                                    ms_sel, ms_idx, vih.shape[1], sih.shape[1]),
+                                    ms_sel, ms_idx, vih.shape[1], sih.shape[1], agg),
         "selected_pairs": int(P_total), "density_vs_causal": round(P_total / (Hq * N * (N + 1) / 2), 5),
         "dense_ms": None if dense_ms is None else round(dense_ms, 3),
         "dense_tflops": None if dense_ms is None else round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
@@ -424,7 +453,7 @@ def run_ours(args, w):
 
 
 def kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, att_bytes, ms_att, ms_sel, ms_idx,
-                     ld_v, ld_s):
+                     ld_v, ld_s, agg=None):
     """Per hot-path kernel: achieved vs the roofline that bounds it.
     attention (+plan, +pack): tensor-bound, 4 d P flops; select x2: HBM-bound,
     4 B per score read + 4 B per index slot written; indexer: fp32 CUDA-core
@@ -440,6 +469,15 @@ def kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, att_bytes, ms_att, m
     out["select_x2"] = {"ms": round(ms_sel, 3), "bound": "hbm",
                         "achieved_gbs": round(sel_bytes / (ms_sel * 1e-3) / 1e9, 1),
                         "frac": round(sel_bytes / (peaks["hbm_gbs"] * 1e9) / (ms_sel * 1e-3), 5)}
+    if agg is not None:
+        # one exp per causal (query, key) pair; MUFU ex2 runs 16 per clock per SM
+        n_exp = Hq * N * (N + 1) / 2
+        mufu_peak = 16 * 148 * peaks.get("sm_max_mhz", 1965.0) * 1e6
+        out["aggregate"] = {"ms": round(agg["ms"], 3), "bound": "alu (MUFU ex2)",
+                            "achieved_gexp_s": round(n_exp / (agg["ms"] * 1e-3) / 1e9, 1),
+                            "peak_gexp_s": round(mufu_peak / 1e9, 1),
+                            "frac": round(n_exp / mufu_peak / (agg["ms"] * 1e-3), 4),
+                            "row_sum_rel_err": agg["row_sum_err"]}
     if w.indexer:
         hidden = w.hidden
         iflops = 2.0 * N * Hkv * (2 * d * hidden + 2 * hidden)

@@ -212,6 +212,32 @@ vs_status vs_dense_attn_fwd(const void* Q, const void* K, const void* V, vs_dtyp
                             cudaStream_t stream);
 
 /*
+ * vs_attn_aggregate -- ground-truth aggregation of the full causal attention
+ * weights along vertical columns and slash diagonals: the indexer's
+ * distillation target (Technical Summary, section 2, "Distillation Training":
+ * a kernel aggregates full attention weights along the columns and diagonals
+ * online during block-wise computation, without the n x n matrix).  For query
+ * head h, with p_ij = exp(scale * q_i . k_j - LSE_i) over j <= i:
+ *     A_v[h][j] = sum_{i >= j} p_ij,    A_s[h][o] = sum_{i >= o} p_{i, i-o},
+ * so each row of A_v and of A_s sums to N (normalise by N for the
+ * distributions the distillation loss compares).
+ *   Q [N, Hq, d], K [N, Hkv, d]: VS_BF16 only (else VS_ERR_UNSUPPORTED);
+ *            d in {64, 128}; strides and GQA as for vs_sparse_attn_fwd.
+ *   lse      fp32 [Hq][N] (device): the row log-sum-exp of the same dense
+ *            causal attention with the same scale, as written by
+ *            vs_dense_attn_fwd.  The weights are only as correct as lse.
+ *   A_v, A_s fp32 [Hq][N] outputs (device).  A_s is zeroed by the call and
+ *            accumulated with fp32 atomics, so its last bits may vary from
+ *            run to run; A_v is written once per entry.
+ *   ws       device workspace of at least 256 bytes, 256-byte aligned (status
+ *            word).
+ */
+vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
+                            int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                            float softmax_scale, const float* lse, float* A_v, float* A_s,
+                            void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Device status of the last call that used `ws`: synchronises `stream`,
  * copies the status word to `*flags` (VS_DEVFLAG_* bits) and returns VS_OK,
  * VS_ERR_DEVICE_TIMEOUT or VS_ERR_DEVICE_BOUNDS accordingly.

@@ -41,6 +41,7 @@ EXPORTS = (
     "vs_status_string", "vs_version", "vs_index_scores", "vs_select_workspace_size", "vs_select",
     "vs_attn_workspace_size", "vs_sparse_attn_fwd", "vs_dense_attn_fwd", "vs_read_device_status",
     "vs_selftest_wait_timeout", "vs_sparse_attn_fwd_static_scratch", "vs_attn_workspace_size_ld",
+    "vs_attn_aggregate",
 )
 
 
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.vs_sparse_attn_fwd.restype = I
         L.vs_dense_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, P, P, P, Z, P]
         L.vs_dense_attn_fwd.restype = I
+        L.vs_attn_aggregate.argtypes = [P, P, I, I, I, I, I, I64, I64, F, P, P, P, P, Z, P]
+        L.vs_attn_aggregate.restype = I
         L.vs_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
         L.vs_read_device_status.restype = I
         L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
@@ -191,6 +194,15 @@ def vs_dense_attn_fwd(Q, K, V, O, lse, ws, softmax_scale=0.0, stream=None):
            "vs_dense_attn_fwd")
 
 
+def vs_attn_aggregate(Q, K, lse, A_v, A_s, ws, softmax_scale=0.0, stream=None):
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    _check(lib().vs_attn_aggregate(_ptr(Q), _ptr(K), _dtype(Q), N, Hq, Hkv, d, Q.stride(0),
+                                   K.stride(0), float(softmax_scale), _ptr(lse), _ptr(A_v),
+                                   _ptr(A_s), _ptr(ws), ws.numel(), _stream(stream)),
+           "vs_attn_aggregate")
+
+
 def vs_read_device_status(ws, stream=None) -> tuple[int, int]:
     """(status code, flags) of the last call that used ``ws`` (synchronises the stream)."""
     flags = ctypes.c_int(0)
@@ -239,3 +251,23 @@ def dense_attention(Q, K, V, ws=None, with_lse=True, stream=None):
     ws = workspace(256, Q.device) if ws is None else ws
     vs_dense_attn_fwd(Q, K, V, O, lse, ws, stream=stream)
     return O, lse
+
+
+def aggregate(Q, K, V=None, lse=None, ws=None, stream=None):
+    """Ground-truth column / diagonal sums (A_v, A_s), fp32 [Hq, N] each.
+
+    Runs the dense causal forward first for the row LSE unless ``lse`` is
+    given (then V is not needed)."""
+    N, Hq, _ = Q.shape
+    ws = ws if ws is not None else workspace(256, Q.device)
+    if lse is None:
+        if V is None:
+            raise ValueError("V is needed to compute the LSE")
+        O = torch.empty_like(Q)
+        lse = torch.empty((Hq, N), dtype=torch.float32, device=Q.device)
+        vs_dense_attn_fwd(Q, K, V, O, lse, ws, stream=stream)
+        del O
+    A_v = torch.empty((Hq, N), dtype=torch.float32, device=Q.device)
+    A_s = torch.empty((Hq, N), dtype=torch.float32, device=Q.device)
+    vs_attn_aggregate(Q, K, lse, A_v, A_s, ws, stream=stream)
+    return A_v, A_s

@@ -226,6 +226,38 @@ vs_status vs_dense_attn_fwd(const void* Q, const void* K, const void* V, vs_dtyp
                    stream);
 }
 
+vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
+                            int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                            float softmax_scale, const float* lse, float* A_v, float* A_s,
+                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!lse || !A_v || !A_s) return VS_ERR_INVALID_ARG;
+  // the checks shared with attention (V and O stand in for K and A_v here)
+  vs_status st = check_attn_common(Q, K, K, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
+                                   softmax_scale, A_v);
+  if (st != VS_OK) return st;
+  if (dtype != VS_BF16) return VS_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < kStatusBytes || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
+  AggArgs a;
+  a.Q = Q;
+  a.K = K;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.q_stride = q_stride_tok;
+  a.kv_stride = kv_stride_tok;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+  a.lse = lse;
+  a.Av = A_v;
+  a.As = A_s;
+  a.status = static_cast<int*>(ws);
+  a.stream = stream;
+  if (cudaMemsetAsync(a.status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  if (cudaMemsetAsync(A_s, 0, sizeof(float) * (size_t)Hq * (size_t)N, stream) != cudaSuccess)
+    return VS_ERR_CUDA;
+  return launch_aggregate(a) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
 vs_status vs_read_device_status(const void* ws, cudaStream_t stream, int* flags) {
   if (!ws || !flags) return VS_ERR_INVALID_ARG;
   int v = 0;

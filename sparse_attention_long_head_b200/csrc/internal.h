@@ -143,6 +143,20 @@ struct AttnArgs {
   void* pack_v;
 };
 
+// Ground-truth aggregation launch description (bf16 Q/K).
+struct AggArgs {
+  const void* Q;
+  const void* K;
+  int N, Hq, Hkv, d;
+  int64_t q_stride, kv_stride;
+  float scale;
+  const float* lse;
+  float* Av;
+  float* As;
+  int* status;
+  cudaStream_t stream;
+};
+
 // Launchers (return a CUDA error; argument checks are done by the caller).
 cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L);
@@ -156,6 +170,7 @@ cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, 
                                 const float* W2, int hidden, float* lv, float* ls,
                                 cudaStream_t stream);
 cudaError_t launch_wait_selftest(int* status, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t launch_aggregate(const AggArgs& a);
 
 // Driver entry point for tensor-map encoding (resolved once through the
 // runtime; no link-time dependency on libcuda).

@@ -128,6 +128,31 @@ def test_attention_host_validation():
     assert rc == vs.VS_ERR_INVALID_ARG
 
 
+def test_aggregate_host_validation():
+    L = vs.lib()
+    f = _fake
+    base = dict(Q=f(0x1000), K=f(0x2000), dtype=0, N=256, Hq=4, Hkv=2, d=128, qs=512, kvs=256,
+                scale=0.0, lse=f(0x3000), Av=f(0x4000), As=f(0x5000), ws=f(0x10000), wsb=256)
+
+    def call(**kw):
+        a = dict(base)
+        a.update(kw)
+        return L.vs_attn_aggregate(a["Q"], a["K"], a["dtype"], a["N"], a["Hq"], a["Hkv"], a["d"],
+                                   a["qs"], a["kvs"], a["scale"], a["lse"], a["Av"], a["As"],
+                                   a["ws"], a["wsb"], None)
+
+    assert call(lse=None) == vs.VS_ERR_INVALID_ARG
+    assert call(Av=None) == vs.VS_ERR_INVALID_ARG
+    assert call(As=None) == vs.VS_ERR_INVALID_ARG
+    assert call(Q=None) == vs.VS_ERR_INVALID_ARG
+    assert call(Hkv=3) == vs.VS_ERR_INVALID_ARG
+    assert call(d=96, qs=384, kvs=192) == vs.VS_ERR_UNSUPPORTED
+    assert call(dtype=1) == vs.VS_ERR_UNSUPPORTED
+    assert call(ws=None) == vs.VS_ERR_WORKSPACE
+    assert call(wsb=100) == vs.VS_ERR_WORKSPACE
+    assert call(N=0) == vs.VS_ERR_INVALID_ARG
+
+
 def test_indexer_and_misc_host_validation():
     L = vs.lib()
     f = _fake
