@@ -34,7 +34,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from vs_workloads import WORKLOADS  # noqa: E402
+from vs_workloads import BATCH_WORKLOADS, WORKLOADS  # noqa: E402
 
 METRIC = "VS-sparse prefill ms/layer & effective TFLOP/s at 128K; speedup vs dense"
 UNIT = "TFLOP/s"
@@ -47,7 +47,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama_128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="llama_128k",
+                    choices=sorted(WORKLOADS) + sorted(BATCH_WORKLOADS))
     ap.add_argument("--dense-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -592,8 +593,259 @@ def run_reference(args, w):
     print(json.dumps(out), flush=True)
 
 
+def batch_oracle_sample(w, Qb, Kb, Vb, sets, seconds, seed=0,
+                        sets_from="this run's GPU selection"):
+    """The fp64 oracle on random rows of random sequences of a batch workload
+    for about `seconds`; effective TFLOP/s by pair count."""
+    import oracle
+    vih, vch, sih, sch = sets
+    cu_h = w.cu_seqlens
+    B, H_sel, Hq, d = len(w.lengths), w.H_sel, w.Hq, w.d
+    rng = np.random.default_rng(seed)
+    t_used, p_done, rows_done = 0.0, 0, 0
+    while t_used < seconds:
+        b = int(rng.integers(0, B))
+        n, t0 = w.lengths[b], int(cu_h[b])
+        h = int(rng.integers(0, Hq))
+        r = b * H_sel + (h * H_sel) // Hq
+        rows = np.sort(rng.integers(0, n, 32))
+        sl = slice(t0, t0 + n)
+        part = slice(b * H_sel, (b + 1) * H_sel)
+        t1 = time.time()
+        oracle.attn_rows(Qb[sl], Kb[sl], Vb[sl], h, rows, vih[part], vch[part], sih[part],
+                         sch[part])
+        t_used += time.time() - t1
+        p_done += int(row_pairs(rows, vih[r, : vch[r]], sih[r, : sch[r]]).sum())
+        rows_done += rows.size
+    return {"value": round(4.0 * d * p_done / t_used / 1e12, 6), "unit": UNIT,
+            "cores": _cpu_cores(), "kind": "oracle",
+            "sample": f"{rows_done} query rows (32 random rows of a random sequence and head per "
+                      f"draw) of {w.name}, fp64 row-form oracle, {t_used:.1f} s; index sets "
+                      f"from {sets_from}"}
+
+
+def run_batch_reference(args, w):
+    """Reference arm of a batch workload: the oracle (its own selection per
+    sequence) on bounded row samples, rank 0 only."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    Qb, Kb, Vb = w.qkv()
+    B, H_sel = len(w.lengths), w.H_sel
+    cap_max = w.cap(max(w.lengths))
+    vih = np.full((B * H_sel, cap_max), -1, np.int32)
+    sih = np.full_like(vih, -1)
+    vch = np.zeros(B * H_sel, np.int32)
+    sch = np.zeros_like(vch)
+    for b, n in enumerate(w.lengths):
+        lv, ls = w.scores(b)
+        k = w.cap(n)
+        vi, vc, _ = oracle.select_heads(lv, w.select_mode_id, k, w.tau_v)
+        si, sc, _ = oracle.select_heads(ls, w.select_mode_id, k, w.tau_s)
+        vih[b * H_sel:(b + 1) * H_sel, :k], vch[b * H_sel:(b + 1) * H_sel] = vi, vc
+        sih[b * H_sel:(b + 1) * H_sel, :k], sch[b * H_sel:(b + 1) * H_sel] = si, sc
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals, last = [], None
+    for it in range(args.warmup + args.steps):
+        last = batch_oracle_sample(w, Qb, Kb, Vb, (vih, vch, sih, sch), per_step, seed=it,
+                                   sets_from="the oracle's own selection")
+        if it >= args.warmup:
+            vals.append(last["value"])
+    value = float(np.mean(vals))
+    print(json.dumps({
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "impl": "reference",
+        "data": "synthetic (seeded generators shaped like the pages' workloads)",
+        "config": {"workload": w.name, "sequences": B, "tokens": int(w.cu_seqlens[-1]),
+                   "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d},
+        "cpu_baseline": dict(last, value=round(value, 6),
+                             sample=last["sample"] + f"; {per_step:.1f} s per step"),
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def run_batch(args, w):
+    """A batch of sequences packed along the token axis: per sequence two
+    selects, then one batched sparse attention call (the step); value =
+    4 d x (selected pairs of every sequence) / step time."""
+    import torch
+    import torch.distributed as dist
+    import sparse_attention_long_head_b200 as vs
+
+    world, rank, local_rank = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    t0 = time.time()
+    Qb, Kb, Vb = w.qkv()
+    scores = [w.scores(b) for b in range(len(w.lengths))]
+    gen_s = time.time() - t0
+    to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    Q, K, V = to_dev(Qb), to_dev(Kb), to_dev(Vb)
+    T, Hq, d = Q.shape
+    B, H_sel, mode = len(w.lengths), w.H_sel, w.select_mode_id
+    cu_h = w.cu_seqlens
+    cu = torch.from_numpy(cu_h).to(dev)
+    max_n = int(max(w.lengths))
+    cap_max = w.cap(max_n)
+    LV = [torch.from_numpy(lv).to(dev) for lv, _ in scores]
+    LS = [torch.from_numpy(ls).to(dev) for _, ls in scores]
+    vi = torch.full((B * H_sel, cap_max), -1, dtype=torch.int32, device=dev)
+    si = torch.full_like(vi, -1)
+    vc = torch.empty(B * H_sel, dtype=torch.int32, device=dev)
+    sc = torch.empty_like(vc)
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=dev)
+    ws_sel = [vs.workspace(vs.vs_select_workspace_size(H_sel, n), dev) for n in w.lengths]
+    ws_att = vs.workspace(vs.vs_attn_workspace_size_varlen(B, max_n, H_sel, d, cap_max), dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = {k: [] for k in ("s0", "a0", "a1")}
+
+    def step(record):
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev["s0"].append(e)
+        for b, n in enumerate(w.lengths):
+            rows = slice(b * H_sel, (b + 1) * H_sel)
+            k = w.cap(n)
+            vs.vs_select(LV[b], mode, k, w.tau_v, vi[rows], vc[rows], ws_sel[b])
+            vs.vs_select(LS[b], mode, k, w.tau_s, si[rows], sc[rows], ws_sel[b])
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev["a0"].append(e)
+        vs.vs_sparse_attn_fwd_varlen(Q, K, V, cu, max_n, vi, vc, si, sc, O, lse, ws_att)
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev["a1"].append(e)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+    rc, flags = vs.vs_read_device_status(ws_att)
+    if rc != vs.VS_OK:
+        raise RuntimeError(f"device status {vs.status_string(rc)} flags {flags}")
+    vih, vch, sih, sch = (x.cpu().numpy() for x in (vi, vc, si, sc))
+    pairs = 0
+    for b, n in enumerate(w.lengths):
+        for h in range(Hq):
+            r = b * H_sel + (h * H_sel) // Hq
+            pairs += pairs_per_set(n, vih[r, : vch[r]], sih[r, : sch[r]])
+    flops = 4.0 * d * pairs
+    dense_pairs = Hq * sum(n * (n + 1) // 2 for n in w.lengths)
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            step(True)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_step = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["s0"], ev["a1"])]))
+    ms_att = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]))
+    ms_step, ms_att = max_over_ranks([ms_step, ms_att], dev)
+    value = whole_job_value(world, flops, ms_step)
+    # dense varlen on the same batch (speed-up denominator)
+    dense_ms = None
+    if args.dense_steps > 0:
+        Od = torch.empty_like(Q)
+        wsd = vs.workspace(256, dev)
+        vs.vs_dense_attn_fwd_varlen(Q, K, V, cu, max_n, Od, None, wsd)
+        ts = []
+        for _ in range(args.dense_steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            vs.vs_dense_attn_fwd_varlen(Q, K, V, cu, max_n, Od, None, wsd)
+            b_.record(stream)
+            b_.synchronize()
+            ts.append(a.elapsed_time(b_))
+        dense_ms = float(np.mean(ts))
+        del Od
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+                      for x in (Qb, Kb, Vb))
+        hS = [torch.from_numpy(x).pin_memory() for pair in scores for x in pair]
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in [hQ, hK, hV] + hS)
+        d2h = hO.numel() * hO.element_size()
+        ts = []
+        for _ in range(2):
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            for b in range(B):
+                LV[b].copy_(hS[2 * b], non_blocking=True)
+                LS[b].copy_(hS[2 * b + 1], non_blocking=True)
+            step(False)
+            hO.copy_(O, non_blocking=True)
+            b_.record(stream)
+            b_.synchronize()
+            ts.append(a.elapsed_time(b_))
+        e2e_ms = max_over_ranks([float(np.min(ts[1:]))], dev)[0]
+        e2e = {"value": round(whole_job_value(world, flops, e2e_ms), 3), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+    peaks, peak_kind = measured_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    algo_bytes = (Q.numel() + K.numel() + V.numel() + O.numel()) * 2 + lse.numel() * 4 \
+        + (vi.numel() + si.numel()) * 4
+    t_roof_ms = max(flops / (peak * 1e12), algo_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generators shaped like the pages' workloads)",
+        "config": {"workload": w.name, "sequences": B, "tokens": int(T), "lengths": list(w.lengths),
+                   "Hq": Hq, "Hkv": w.Hkv, "d": d, "H_sel": H_sel, "select": w.select_mode,
+                   "cap_frac": w.cap_frac, "tau_v": w.tau_v, "tau_s": w.tau_s,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "a 256 MiB buffer is written between timed steps, outside the timed "
+                         "windows"},
+        "ms_select": round(ms_step - ms_att, 3), "ms_attention": round(ms_att, 3),
+        "selected_pairs": int(pairs), "density_vs_causal": round(pairs / dense_pairs, 5),
+        "dense_ms": None if dense_ms is None else round(dense_ms, 3),
+        "speedup_vs_dense": None if dense_ms is None else round(dense_ms / ms_step, 3),
+        "roofline": {"bound": "tensor", "achieved": round(flops / (ms_att * 1e-3) / 1e12, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(t_roof_ms / ms_att, 4),
+                     "traffic": None, "kernel": "vs_sparse_attn_fwd_varlen (plan + pack + attn)",
+                     "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)"},
+        "e2e": e2e, "gpu_launches": (2 * B + 3) * args.steps, "input_gen_s": round(gen_s, 1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = batch_oracle_sample(w, Qb, Kb, Vb, (vih, vch, sih, sch),
+                                                  args.cpu_seconds)
+    out["clocks"] = clk.summary()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
+    if args.workload in BATCH_WORKLOADS:
+        if args.impl == "reference":
+            run_batch_reference(args, BATCH_WORKLOADS[args.workload])
+        else:
+            run_batch(args, BATCH_WORKLOADS[args.workload])
+        return
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)

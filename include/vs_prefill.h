@@ -169,6 +169,45 @@ vs_status vs_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dty
                              size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * vs_sparse_attn_fwd_varlen / vs_dense_attn_fwd_varlen -- the same attention
+ * over a batch of B independent sequences packed along the token axis
+ * (variable-length batched prefill; each sequence attends only to itself).
+ *   total_tokens  rows of Q, K, V, O (and columns of lse: lse is fp32
+ *            [Hq][total_tokens]); at most 2^31 - 1.
+ *   cu_seqlens    int32 [B + 1] (DEVICE): sequence b is tokens
+ *            [cu_seqlens[b], cu_seqlens[b + 1]); the offsets must not
+ *            decrease, start at >= 0, end at <= total_tokens and give no
+ *            sequence longer than max_seqlen.  A malformed entry makes that
+ *            sequence empty (its O rows are not written) and sets
+ *            VS_DEVFLAG_BOUNDS.
+ *   max_seqlen    the longest sequence (sizes the plan; >= 1).
+ *   Index sets (sparse): one per (sequence, index-set head): v_idx
+ *            [B * H_sel][v_ld] with v_cnt [B * H_sel] (row b * H_sel + hs),
+ *            likewise s_idx / s_cnt; positions are relative to the sequence
+ *            start (columns and offsets in [0, that sequence's length)).
+ *   ws       at least vs_attn_workspace_size_varlen(B, max_seqlen, H_sel, d,
+ *            0) bytes (the plan; dense: 256); with v_ld in place of 0, room to
+ *            pack the selected vertical rows, as for vs_sparse_attn_fwd.
+ *   VS_BF16 only (else VS_ERR_UNSUPPORTED); B * H_sel <= 65535.
+ * The pages prefill one sequence at a time; this batching follows their
+ * per-sequence definition unchanged.
+ */
+size_t vs_attn_workspace_size_varlen(int B, int max_seqlen, int H_sel, int d, int64_t v_ld);
+vs_status vs_sparse_attn_fwd_varlen(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                    int total_tokens, int B, const int32_t* cu_seqlens,
+                                    int max_seqlen, int Hq, int Hkv, int d, int64_t q_stride_tok,
+                                    int64_t kv_stride_tok, float softmax_scale, int H_sel,
+                                    const int32_t* v_idx, int64_t v_ld, const int32_t* v_cnt,
+                                    const int32_t* s_idx, int64_t s_ld, const int32_t* s_cnt,
+                                    void* O, float* lse, void* ws, size_t ws_bytes,
+                                    cudaStream_t stream);
+vs_status vs_dense_attn_fwd_varlen(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                   int total_tokens, int B, const int32_t* cu_seqlens,
+                                   int max_seqlen, int Hq, int Hkv, int d, int64_t q_stride_tok,
+                                   int64_t kv_stride_tok, float softmax_scale, void* O, float* lse,
+                                   void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * vs_sparse_attn_fwd_static_scratch -- vs_sparse_attn_fwd without a
  * caller-provided workspace.  The summary pages have no counterpart to this
  * call; it exists for callers that cannot allocate device memory: plain-C

@@ -41,7 +41,8 @@ EXPORTS = (
     "vs_status_string", "vs_version", "vs_index_scores", "vs_select_workspace_size", "vs_select",
     "vs_attn_workspace_size", "vs_sparse_attn_fwd", "vs_dense_attn_fwd", "vs_read_device_status",
     "vs_selftest_wait_timeout", "vs_sparse_attn_fwd_static_scratch", "vs_attn_workspace_size_ld",
-    "vs_attn_aggregate",
+    "vs_attn_aggregate", "vs_attn_workspace_size_varlen", "vs_sparse_attn_fwd_varlen",
+    "vs_dense_attn_fwd_varlen",
 )
 
 
@@ -86,6 +87,14 @@ def lib() -> ctypes.CDLL:
         L.vs_dense_attn_fwd.restype = I
         L.vs_attn_aggregate.argtypes = [P, P, I, I, I, I, I, I64, I64, F, P, P, P, P, Z, P]
         L.vs_attn_aggregate.restype = I
+        L.vs_attn_workspace_size_varlen.argtypes = [I, I, I, I, I64]
+        L.vs_attn_workspace_size_varlen.restype = Z
+        L.vs_sparse_attn_fwd_varlen.argtypes = [P, P, P, I, I, I, P, I, I, I, I, I64, I64, F, I, P,
+                                                I64, P, P, I64, P, P, P, P, Z, P]
+        L.vs_sparse_attn_fwd_varlen.restype = I
+        L.vs_dense_attn_fwd_varlen.argtypes = [P, P, P, I, I, I, P, I, I, I, I, I64, I64, F, P, P,
+                                               P, Z, P]
+        L.vs_dense_attn_fwd_varlen.restype = I
         L.vs_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
         L.vs_read_device_status.restype = I
         L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
@@ -140,6 +149,10 @@ def vs_attn_workspace_size(N: int, Hq: int, H_sel: int, d: int) -> int:
 
 def vs_attn_workspace_size_ld(N: int, Hq: int, H_sel: int, d: int, v_ld: int) -> int:
     return lib().vs_attn_workspace_size_ld(N, Hq, H_sel, d, v_ld)
+
+
+def vs_attn_workspace_size_varlen(B: int, max_seqlen: int, H_sel: int, d: int, v_ld: int = 0) -> int:
+    return int(lib().vs_attn_workspace_size_varlen(B, max_seqlen, H_sel, d, v_ld))
 
 
 def vs_index_scores(K, V, W1, W2, logits_v, logits_s, stream=None):
@@ -201,6 +214,30 @@ def vs_attn_aggregate(Q, K, lse, A_v, A_s, ws, softmax_scale=0.0, stream=None):
                                    K.stride(0), float(softmax_scale), _ptr(lse), _ptr(A_v),
                                    _ptr(A_s), _ptr(ws), ws.numel(), _stream(stream)),
            "vs_attn_aggregate")
+
+
+def vs_sparse_attn_fwd_varlen(Q, K, V, cu_seqlens, max_seqlen, v_idx, v_cnt, s_idx, s_cnt, O, lse,
+                              ws, softmax_scale=0.0, stream=None):
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    H_sel = v_idx.shape[0] // B
+    _check(lib().vs_sparse_attn_fwd_varlen(
+        _ptr(Q), _ptr(K), _ptr(V), _dtype(Q), T, B, _ptr(cu_seqlens), int(max_seqlen), Hq, Hkv, d,
+        Q.stride(0), K.stride(0), float(softmax_scale), H_sel, _ptr(v_idx), v_idx.stride(0),
+        _ptr(v_cnt), _ptr(s_idx), s_idx.stride(0), _ptr(s_cnt), _ptr(O), _ptr(lse), _ptr(ws),
+        ws.numel(), _stream(stream)), "vs_sparse_attn_fwd_varlen")
+
+
+def vs_dense_attn_fwd_varlen(Q, K, V, cu_seqlens, max_seqlen, O, lse, ws, softmax_scale=0.0,
+                             stream=None):
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    _check(lib().vs_dense_attn_fwd_varlen(
+        _ptr(Q), _ptr(K), _ptr(V), _dtype(Q), T, B, _ptr(cu_seqlens), int(max_seqlen), Hq, Hkv, d,
+        Q.stride(0), K.stride(0), float(softmax_scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream(stream)), "vs_dense_attn_fwd_varlen")
 
 
 def vs_read_device_status(ws, stream=None) -> tuple[int, int]:

@@ -1,6 +1,7 @@
 // C ABI of libvs: argument validation, workspace layout and launches.
 // Declarations and their documentation: include/vs_prefill.h.
 #include <cmath>
+#include <cstdint>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -147,6 +148,7 @@ size_t vs_attn_workspace_size(int N, int Hq, int H_sel, int d) {
 }
 
 static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
+                           int B, int64_t total, const int32_t* cu_seqlens,
                            int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
                            float softmax_scale, bool sparse, int H_sel, const int32_t* v_idx,
                            int64_t v_ld, const int32_t* v_cnt, const int32_t* s_idx, int64_t s_ld,
@@ -162,7 +164,10 @@ static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype
   } else {
     H_sel = 1;
   }
-  const PlanLayout L = PlanLayout::make(N, H_sel);
+  if (B < 1 || total < 1 || total > INT32_MAX || (B > 1 && !cu_seqlens)) return VS_ERR_INVALID_ARG;
+  if (cu_seqlens && dtype != VS_BF16) return VS_ERR_UNSUPPORTED;  // batches: tensor-core path
+  if ((int64_t)B * H_sel > 65535) return VS_ERR_UNSUPPORTED;
+  const PlanLayout L = PlanLayout::make(N, B * H_sel);
   const size_t need = sparse ? L.total : kStatusBytes;  // the plan alone suffices
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
   AttnArgs a;
@@ -176,6 +181,9 @@ static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype
   a.Hkv = Hkv;
   a.d = d;
   a.H_sel = H_sel;
+  a.B = B;
+  a.total = total;
+  a.cu_seqlens = cu_seqlens;
   a.q_stride = q_stride_tok;
   a.kv_stride = kv_stride_tok;
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
@@ -192,7 +200,7 @@ static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype
   a.pack_vrows = 0;
   a.pack_k = a.pack_v = nullptr;
   if (sparse && dtype == VS_BF16 && PackedLayout::eligible(Hq, Hkv, H_sel)) {
-    const PackedLayout Pk = PackedLayout::make(L, H_sel, d, v_ld);
+    const PackedLayout Pk = PackedLayout::make(L, B * H_sel, d, v_ld);
     if (ws_bytes >= Pk.offset + Pk.bytes) {  // room to pack the vertical rows
       a.pack_vrows = Pk.vrows;
       a.pack_k = static_cast<char*>(ws) + Pk.offset;
@@ -212,18 +220,51 @@ vs_status vs_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dty
                              const int32_t* v_cnt, const int32_t* s_idx, int64_t s_ld,
                              const int32_t* s_cnt, void* O, float* lse, void* ws,
                              size_t ws_bytes, cudaStream_t stream) {
-  return attn_impl(Q, K, V, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok, softmax_scale,
-                   true, H_sel, v_idx, v_ld, v_cnt, s_idx, s_ld, s_cnt, O, lse, ws, ws_bytes,
-                   stream);
+  return attn_impl(Q, K, V, dtype, N, 1, N, nullptr, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
+                   softmax_scale, true, H_sel, v_idx, v_ld, v_cnt, s_idx, s_ld, s_cnt, O, lse,
+                   ws, ws_bytes, stream);
+}
+
+size_t vs_attn_workspace_size_varlen(int B, int max_seqlen, int H_sel, int d, int64_t v_ld) {
+  if (B < 1 || max_seqlen < 1 || H_sel < 1 || (d != 64 && d != 128)) return kStatusBytes;
+  const PlanLayout L = PlanLayout::make(max_seqlen, B * H_sel);
+  if (v_ld < 1) return L.total;
+  const PackedLayout Pk = PackedLayout::make(L, B * H_sel, d, v_ld);
+  return Pk.offset + Pk.bytes;
+}
+
+vs_status vs_sparse_attn_fwd_varlen(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                    int total_tokens, int B, const int32_t* cu_seqlens,
+                                    int max_seqlen, int Hq, int Hkv, int d, int64_t q_stride_tok,
+                                    int64_t kv_stride_tok, float softmax_scale, int H_sel,
+                                    const int32_t* v_idx, int64_t v_ld, const int32_t* v_cnt,
+                                    const int32_t* s_idx, int64_t s_ld, const int32_t* s_cnt,
+                                    void* O, float* lse, void* ws, size_t ws_bytes,
+                                    cudaStream_t stream) {
+  if (!cu_seqlens) return VS_ERR_INVALID_ARG;
+  return attn_impl(Q, K, V, dtype, max_seqlen, B, total_tokens, cu_seqlens, Hq, Hkv, d,
+                   q_stride_tok, kv_stride_tok, softmax_scale, true, H_sel, v_idx, v_ld, v_cnt,
+                   s_idx, s_ld, s_cnt, O, lse, ws, ws_bytes, stream);
+}
+
+vs_status vs_dense_attn_fwd_varlen(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                   int total_tokens, int B, const int32_t* cu_seqlens,
+                                   int max_seqlen, int Hq, int Hkv, int d, int64_t q_stride_tok,
+                                   int64_t kv_stride_tok, float softmax_scale, void* O, float* lse,
+                                   void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!cu_seqlens) return VS_ERR_INVALID_ARG;
+  return attn_impl(Q, K, V, dtype, max_seqlen, B, total_tokens, cu_seqlens, Hq, Hkv, d,
+                   q_stride_tok, kv_stride_tok, softmax_scale, false, 1, nullptr, 0, nullptr,
+                   nullptr, 0, nullptr, O, lse, ws, ws_bytes, stream);
 }
 
 vs_status vs_dense_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype, int N,
                             int Hq, int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
                             float softmax_scale, void* O, float* lse, void* ws, size_t ws_bytes,
                             cudaStream_t stream) {
-  return attn_impl(Q, K, V, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok, softmax_scale,
-                   false, 1, nullptr, 0, nullptr, nullptr, 0, nullptr, O, lse, ws, ws_bytes,
-                   stream);
+  return attn_impl(Q, K, V, dtype, N, 1, N, nullptr, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
+                   softmax_scale, false, 1, nullptr, 0, nullptr, nullptr, 0, nullptr, O, lse, ws,
+                   ws_bytes, stream);
 }
 
 vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,

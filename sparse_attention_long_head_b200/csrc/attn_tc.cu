@@ -76,7 +76,9 @@ __device__ int block_bits_to_list(const uint32_t* bits, int64_t nwords, int64_t 
 }
 
 struct PlanKernelArgs {
-  int N, H_sel;
+  int N, H_sel;  // N: the longest sequence; slots are b * H_sel + hs
+  const int32_t* cu;
+  int64_t total;
   const int32_t* v_idx;
   int64_t v_ld;
   const int32_t* v_cnt;
@@ -95,17 +97,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanKernelArgs a) {
   __shared__ uint32_t dbits[1026];  // touched block-diagonals, T <= 32768
   __shared__ uint32_t d1bits[1026];
   __shared__ int bad;
-  const int hs = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+  const int hs = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;  // hs: the plan slot
   const PlanLayout& L = a.L;
   PlanPtrs pp = plan_ptrs(L, a.ws);
   uint32_t* vb = pp.vbits + (int64_t)hs * L.vbits_words;
   uint32_t* sb = pp.sbits + (int64_t)hs * L.sbits_words;
-  const int N = a.N, T = L.T;
+  int64_t tok0;
+  int N;
+  const bool seq_ok = seq_range(a.cu, a.total, a.N, hs / a.H_sel, tok0, N);
+  const int T = (N + 127) / 128;
   const int dwords = (T + 2 + 31) / 32;
   for (int64_t w = tid; w < L.vbits_words; w += nt) vb[w] = 0;
   for (int64_t w = tid; w < L.sbits_words; w += nt) sb[w] = 0;
   for (int w = tid; w < dwords; w += nt) dbits[w] = 0;
-  if (tid == 0) bad = 0;
+  if (tid == 0) bad = seq_ok ? 0 : 1;
   __syncthreads();
 
   int nv_in = a.v_cnt[hs], ns_in = a.s_cnt[hs];
@@ -142,8 +147,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanKernelArgs a) {
     d1bits[w] = cur | (cur << 1) | (prev >> 31);
   }
   __syncthreads();
-  int32_t* vlist = pp.vlist + (int64_t)hs * N;
-  int32_t* slist = pp.slist + (int64_t)hs * N;
+  int32_t* vlist = pp.vlist + (int64_t)hs * L.N;
+  int32_t* slist = pp.slist + (int64_t)hs * L.N;
   int32_t* d1list = pp.d1list + (int64_t)hs * L.d1_len;
   int32_t* d1pref = pp.d1pref + (int64_t)hs * L.d1pref_len;
   int32_t* vpair = pp.vpair + (int64_t)hs * L.vpair_len;
@@ -195,8 +200,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanKernelArgs a) {
 
 cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L) {
   if (L.T + 2 > 1026 * 32) return cudaErrorInvalidValue;
-  PlanKernelArgs k{a.N, a.H_sel, a.v_idx, a.v_ld, a.v_cnt, a.s_idx, a.s_ld, a.s_cnt, a.ws, a.status, L};
-  plan_kernel<<<a.H_sel, kPlanThreads, 0, a.stream>>>(k);
+  PlanKernelArgs k{a.N,   a.H_sel, a.cu_seqlens, a.total, a.v_idx, a.v_ld, a.v_cnt,
+                   a.s_idx, a.s_ld,  a.s_cnt,      a.ws,    a.status, L};
+  plan_kernel<<<a.B * a.H_sel, kPlanThreads, 0, a.stream>>>(k);
   return cudaGetLastError();
 }
 
@@ -209,11 +215,15 @@ template <int D>
 __global__ void __launch_bounds__(256) pack_kernel(const __nv_bfloat16* K, const __nv_bfloat16* V,
                                                    int64_t kv_stride, int Hq, int Hkv, int H_sel,
                                                    int64_t vrows, PlanLayout L, PlanPtrs pp,
+                                                   const int32_t* cu, int64_t total,
                                                    __nv_bfloat16* pk, __nv_bfloat16* pv) {
-  const int hs = blockIdx.y, c = blockIdx.x;
+  const int hs = blockIdx.y, c = blockIdx.x;  // hs: the plan slot
   const int nv = pp.meta[4 * hs + 0];
   if (128 * c >= nv) return;
-  const int g = (hs * (Hq / H_sel)) / (Hq / Hkv);
+  int64_t tok0;
+  int Nb;
+  seq_range(cu, total, L.N, hs / H_sel, tok0, Nb);  // nv == 0 for a malformed entry
+  const int g = ((hs % H_sel) * (Hq / H_sel)) / (Hq / Hkv);
   const int32_t* vl = pp.vlist + (int64_t)hs * L.N;
   constexpr int CH = D / 8;  // 16-byte chunks per row
   for (int e = threadIdx.x; e < 128 * CH; e += blockDim.x) {
@@ -221,7 +231,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const __nv_bfloat16* K, const
     const int t = 128 * c + r;
     uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
     if (t < nv) {
-      const int64_t src = (int64_t)vl[t] * kv_stride + (int64_t)g * D + ch * 8;
+      const int64_t src = (tok0 + vl[t]) * kv_stride + (int64_t)g * D + ch * 8;
       kk = *reinterpret_cast<const uint4*>(K + src);
       vv = *reinterpret_cast<const uint4*>(V + src);
     }
@@ -232,7 +242,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const __nv_bfloat16* K, const
 }
 
 cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L) {
-  dim3 grid((unsigned)(a.pack_vrows / 128), (unsigned)a.H_sel);
+  dim3 grid((unsigned)(a.pack_vrows / 128), (unsigned)(a.B * a.H_sel));
   const PlanPtrs pp = plan_ptrs(L, a.ws);
   auto* K = static_cast<const __nv_bfloat16*>(a.K);
   auto* V = static_cast<const __nv_bfloat16*>(a.V);
@@ -240,10 +250,10 @@ cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L) {
   auto* pv = static_cast<__nv_bfloat16*>(a.pack_v);
   if (a.d == 128)
     pack_kernel<128><<<grid, 256, 0, a.stream>>>(K, V, a.kv_stride, a.Hq, a.Hkv, a.H_sel,
-                                                 a.pack_vrows, L, pp, pk, pv);
+                                                 a.pack_vrows, L, pp, a.cu_seqlens, a.total, pk, pv);
   else
     pack_kernel<64><<<grid, 256, 0, a.stream>>>(K, V, a.kv_stride, a.Hq, a.Hkv, a.H_sel,
-                                                a.pack_vrows, L, pp, pk, pv);
+                                                a.pack_vrows, L, pp, a.cu_seqlens, a.total, pk, pv);
   return cudaGetLastError();
 }
 
@@ -267,8 +277,11 @@ struct Cfg {
 };
 
 struct AttnParams {
-  int N, Hq, Hkv, H_sel, T, P, G;
-  int num_units;
+  int N, Hq, Hkv, H_sel, T, P, G;  // N, T, P: of the longest sequence
+  int num_units;                   // B * Hq * P
+  const int32_t* cu;               // sequence offsets (device) or null
+  int B;                           // sequences
+  int64_t total;                   // token rows of Q, K, V, O
   int64_t q_stride;
   float scale_log2;  // softmax scale * log2(e)
   __nv_bfloat16* O;
@@ -281,25 +294,46 @@ struct AttnParams {
 };
 
 struct UnitInfo {
-  int h, hs, g, p, n, mode, nvc, nv, d1start;
+  int h, hs, g, p, n, mode, nvc, nv, d1start;  // hs: the plan slot b * H_sel + index set
+  int b;                                        // the unit's sequence
+  int Nb;                                       // its tokens
 };
+
+// First token row of the unit's sequence (re-read where needed rather than
+// kept live through the tile loop).
+__device__ __forceinline__ int64_t unit_tok0(const AttnParams& P, const UnitInfo& ui) {
+  return P.cu ? (int64_t)__ldg(P.cu + ui.b) : 0;
+}
 
 template <bool SPARSE>
 __device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
   // Units grouped by KV head (so CTAs running at the same time stream the same
   // K/V and share it in L2), heaviest (largest p) first within a group, the G
   // query heads of a group adjacent.
+  // Sequences of a batch come one after another.
   UnitInfo ui;
+  const int per_seq = P.Hq * P.P;
+  const int bseq = u / per_seq;
+  u -= bseq * per_seq;
+  int64_t tok0_unused;
+  seq_range(P.cu, P.total, P.N, bseq, tok0_unused, ui.Nb);
+  ui.b = bseq;
   ui.g = u / (P.G * P.P);
   const int rem = u - ui.g * P.G * P.P;
   ui.p = P.P - 1 - rem / P.G;
   ui.h = ui.g * P.G + rem % P.G;
-  ui.hs = (int)(((int64_t)ui.h * P.H_sel) / P.Hq);
-  const int last_b = min(2 * ui.p + 1, P.T - 1);
-  const int n_dense = last_b + 1;
+  ui.hs = bseq * P.H_sel + (int)(((int64_t)ui.h * P.H_sel) / P.Hq);
+  const int Tb = (ui.Nb + 127) / 128;
+  const int last_b = min(2 * ui.p + 1, Tb - 1);
+  const int n_dense = max(0, last_b + 1);  // 0: the pair lies past the sequence's end
   ui.nvc = 0;
   ui.nv = 0;
   ui.d1start = 0;
+  if (n_dense == 0) {
+    ui.mode = kModeDense;
+    ui.n = 0;
+    return ui;
+  }
   if (!SPARSE) {
     ui.mode = kModeDense;
     ui.n = n_dense;
@@ -355,7 +389,7 @@ template <bool SPARSE>
 __device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& ui, const Item& it,
                                           int i, int t_sub, uint32_t (&w)[4]) {
   if (it.kind == kItemVChunk) {
-    const int32_t* base = P.pp.vlist + (int64_t)ui.hs * P.N + 128 * it.b;
+    const int32_t* base = P.pp.vlist + (int64_t)ui.hs * P.L.N + 128 * it.b;
     const int cnt = min(128, ui.nv - 128 * it.b);
     int n = cnt;
     if (base[cnt - 1] > i) {
@@ -384,7 +418,7 @@ __device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& u
   }
   // offset window: bit c = [ i - (128 b + c) is a selected offset ]
   const uint32_t* sb = P.pp.sbits + (int64_t)ui.hs * P.L.sbits_words;
-  const int64_t pos0 = (int64_t)P.N - i + 128 + 128 * b;
+  const int64_t pos0 = (int64_t)ui.Nb - i + 128 + 128 * b;
   const uint32_t* sw = sb + (pos0 >> 5);
   const int sh = (int)(pos0 & 31);
   uint32_t x[5];
@@ -529,6 +563,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tslot;
   const WaitCtx wc{P.wait_limit_ns, P.status, abort_flag};
+  if (!SPARSE && P.cu && blockIdx.x == 0 && tid == 0) {
+    // the sparse path's plan kernel checks the offsets; here the first CTA does
+    for (int b = 0; b < P.B; ++b) {
+      int64_t t0;
+      int nb;
+      if (!seq_range(P.cu, P.total, P.N, b, t0, nb)) atomicOr(P.status, VS_DEVFLAG_BOUNDS);
+    }
+  }
 
   if (warp < 8) {
     // ------------------------------------------------ softmax + epilogue
@@ -542,14 +584,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
       const UnitInfo ui = unit_info<SPARSE>(P, u);
       const int i = 256 * ui.p + 128 * sub + r;
-      const int im = min(i, P.N - 1);
+      const int im = max(0, min(i, ui.Nb - 1));
       const int t_sub = 2 * ui.p + sub;
-      __nv_bfloat16* orow = P.O + (int64_t)i * P.q_stride + (int64_t)ui.h * D;
+      // output row pointers are formed where they are used (few live registers
+      // across the tile loop)
+      auto orow_of = [&]() {
+        return P.O + (unit_tok0(P, ui) + i) * P.q_stride + (int64_t)ui.h * D;
+      };
+      auto lrow_of = [&]() { return P.lse + (int64_t)ui.h * P.total + unit_tok0(P, ui) + i; };
       if (ui.n == 0) {
-        if (i < P.N) {
+        if (i < ui.Nb) {
+          __nv_bfloat16* orow = orow_of();
           for (int c = 0; c < D; c += 8)
             *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-          if (P.lse) P.lse[(int64_t)ui.h * P.N + i] = -INFINITY;
+          if (P.lse) *lrow_of() = -INFINITY;
         }
         continue;
       }
@@ -623,12 +671,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!mbar_wait(bar(B_OFULL + sub), ucount & 1, wc)) { ok = false; break; }
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = orow_of();
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * q, o);
         tmem_ld_wait(o);
-        if (i < P.N) {
+        if (i < ui.Nb) {
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
             uint4 v;
@@ -640,8 +689,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      if (i < P.N && P.lse)
-        P.lse[(int64_t)ui.h * P.N + i] =
+      if (i < ui.Nb && P.lse)
+        *lrow_of() =
             l > 0.f ? (m_use + log2f(l)) * 0.6931471805599453f : -INFINITY;
       ++ucount;
     }
@@ -735,12 +784,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const UnitInfo ui = unit_info<SPARSE>(P, u);
       if (ui.n == 0) continue;
       if (ucount > 0 && !mbar_wait(bar(B_QEMPTY), (ucount - 1) & 1, wc)) { ok = false; break; }
+      const int64_t tok0 = unit_tok0(P, ui);
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kQBytes);
         for (int s = 0; s < 2; ++s)
           for (int h = 0; h < nsub64; ++h)
             tma_load_2d(smem_u32(sQ + s * C::kQBytes + h * 16384), &tmQ, bar(B_QFULL),
-                        ui.h * D + 64 * h, 256 * ui.p + 128 * s);
+                        ui.h * D + 64 * h, (int)(tok0 + 256 * ui.p + 128 * s));
       }
       ++ucount;
       // tile t of the unit: K(t/2) for even t, V(t/2) for odd t; a stage
@@ -767,7 +817,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (lane == 0) {
               const CUtensorMap* m = kv ? &tmV : &tmK;
               for (int h = 0; h < nsub64; ++h)
-                tma_load_2d(dst + h * 16384, m, fb, ui.g * D + 64 * h, 128 * it.b);
+                tma_load_2d(dst + h * 16384, m, fb, ui.g * D + 64 * h, (int)(tok0 + 128 * it.b));
             }
           } else if (P.pack_vrows > 0) {
             if (lane == 0) {
@@ -777,13 +827,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             (int)(ui.hs * P.pack_vrows + 128 * it.b));
             }
           } else {
-            const int32_t* base = P.pp.vlist + (int64_t)ui.hs * P.N + 128 * it.b;
+            const int32_t* base = P.pp.vlist + (int64_t)ui.hs * P.L.N + 128 * it.b;
             const int cnt = min(128, ui.nv - 128 * it.b);
             int rr[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int e = 4 * lane + q;
-              rr[q] = base[e < cnt ? e : 0];
+              rr[q] = (int)tok0 + base[e < cnt ? e : 0];
             }
             const CUtensorMap* m = kv ? &tmVg : &tmKg;
             for (int h = 0; h < nsub64; ++h)
@@ -832,15 +882,15 @@ static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap mQ, mK, mV, mKg, mVg;
   CUresult rc = CUDA_SUCCESS;
-  encode_map(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.N, a.q_stride, 128, &rc);
-  encode_map(enc, &mK, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, 128, &rc);
-  encode_map(enc, &mV, a.V, (int64_t)a.Hkv * D, a.N, a.kv_stride, 128, &rc);
+  encode_map(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.total, a.q_stride, 128, &rc);
+  encode_map(enc, &mK, a.K, (int64_t)a.Hkv * D, a.total, a.kv_stride, 128, &rc);
+  encode_map(enc, &mV, a.V, (int64_t)a.Hkv * D, a.total, a.kv_stride, 128, &rc);
   if (SPARSE && a.pack_vrows > 0) {  // packed vertical rows: [H_sel * vrows][D] tiles
-    encode_map(enc, &mKg, a.pack_k, D, (int64_t)a.H_sel * a.pack_vrows, D, 128, &rc);
-    encode_map(enc, &mVg, a.pack_v, D, (int64_t)a.H_sel * a.pack_vrows, D, 128, &rc);
+    encode_map(enc, &mKg, a.pack_k, D, (int64_t)a.B * a.H_sel * a.pack_vrows, D, 128, &rc);
+    encode_map(enc, &mVg, a.pack_v, D, (int64_t)a.B * a.H_sel * a.pack_vrows, D, 128, &rc);
   } else {
-    encode_map(enc, &mKg, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
-    encode_map(enc, &mVg, a.V, (int64_t)a.Hkv * D, a.N, a.kv_stride, 1, &rc);
+    encode_map(enc, &mKg, a.K, (int64_t)a.Hkv * D, a.total, a.kv_stride, 1, &rc);
+    encode_map(enc, &mVg, a.V, (int64_t)a.Hkv * D, a.total, a.kv_stride, 1, &rc);
   }
   if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
   AttnParams P;
@@ -851,7 +901,10 @@ static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
   P.T = L.T;
   P.P = L.P;
   P.G = a.Hq / a.Hkv;
-  P.num_units = a.Hq * L.P;
+  P.num_units = a.B * a.Hq * L.P;
+  P.cu = a.cu_seqlens;
+  P.B = a.B;
+  P.total = a.total;
   P.q_stride = a.q_stride;
   P.scale_log2 = a.scale * 1.4426950408889634f;
   P.O = static_cast<__nv_bfloat16*>(a.O);

@@ -117,14 +117,41 @@ struct PackedLayout {
   }
 };
 
-// Common attention launch description.
+// Sequence b of a packed batch: tokens [tok0, tok0 + Nb) of every tensor.
+// Without cu_seqlens the batch is one sequence of maxN tokens.  A malformed
+// entry (negative, decreasing, past `total` or longer than maxN) gives an
+// empty sequence and returns false (callers flag VS_DEVFLAG_BOUNDS).
+__host__ __device__ inline bool seq_range(const int32_t* cu, int64_t total, int maxN, int b,
+                                          int64_t& tok0, int& Nb) {
+  if (!cu) {
+    tok0 = 0;
+    Nb = maxN;
+    return true;
+  }
+  const int64_t s = cu[b], e = cu[b + 1];
+  if (s < 0 || e < s || e > total || e - s > maxN) {
+    tok0 = 0;
+    Nb = 0;
+    return false;
+  }
+  tok0 = s;
+  Nb = static_cast<int>(e - s);
+  return true;
+}
+
+// Common attention launch description.  A batch of B sequences packed along
+// the token axis (cu_seqlens, device, B + 1 offsets; null for one sequence)
+// has plan slots b * H_sel + hs, each laid out for N = the longest sequence.
 struct AttnArgs {
   const void* Q;
   const void* K;
   const void* V;
   void* O;
   float* lse;
-  int N, Hq, Hkv, d, H_sel;
+  int N, Hq, Hkv, d, H_sel;  // N: the longest sequence (the only one when B = 1)
+  int B;                     // sequences
+  int64_t total;             // token rows of Q, K, V, O (= N when B = 1)
+  const int32_t* cu_seqlens; // device [B + 1] or null
   int64_t q_stride, kv_stride;
   float scale;
   bool sparse;

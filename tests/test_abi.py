@@ -128,6 +128,41 @@ def test_attention_host_validation():
     assert rc == vs.VS_ERR_INVALID_ARG
 
 
+def test_varlen_host_validation():
+    L = vs.lib()
+    f = _fake
+    base = dict(Q=f(0x1000), K=f(0x2000), V=f(0x3000), dtype=0, T=1000, B=3, cu=f(0x9000),
+                maxn=500, Hq=4, Hkv=2, d=128, qs=512, kvs=256, scale=0.0, Hsel=2, vi=f(0x4000),
+                vld=8, vc=f(0x5000), si=f(0x6000), sld=8, sc=f(0x7000), O=f(0x8000), lse=None,
+                ws=f(0x10000), wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(base)
+        a.update(kw)
+        return L.vs_sparse_attn_fwd_varlen(a["Q"], a["K"], a["V"], a["dtype"], a["T"], a["B"],
+                                           a["cu"], a["maxn"], a["Hq"], a["Hkv"], a["d"], a["qs"],
+                                           a["kvs"], a["scale"], a["Hsel"], a["vi"], a["vld"],
+                                           a["vc"], a["si"], a["sld"], a["sc"], a["O"], a["lse"],
+                                           a["ws"], a["wsb"], None)
+
+    assert call(cu=None) == vs.VS_ERR_INVALID_ARG
+    assert call(B=0) == vs.VS_ERR_INVALID_ARG
+    assert call(T=0) == vs.VS_ERR_INVALID_ARG
+    assert call(maxn=0) == vs.VS_ERR_INVALID_ARG
+    assert call(dtype=1) == vs.VS_ERR_UNSUPPORTED
+    assert call(Hsel=3) == vs.VS_ERR_INVALID_ARG
+    assert call(wsb=1000) == vs.VS_ERR_WORKSPACE
+    rc = L.vs_dense_attn_fwd_varlen(f(), f(), f(), 0, 100, 2, None, 50, 1, 1, 64, 64, 64, 0.0,
+                                    f(), None, f(0x10000), 256, None)
+    assert rc == vs.VS_ERR_INVALID_ARG
+    # the plan grows with the batch; packing needs room for every slot
+    one = vs.vs_attn_workspace_size_varlen(1, 4096, 4, 128, 0)
+    assert one == vs.vs_attn_workspace_size(4096, 4, 4, 128)
+    assert vs.vs_attn_workspace_size_varlen(3, 4096, 4, 128, 0) > 2 * one
+    assert vs.vs_attn_workspace_size_varlen(3, 4096, 4, 128, 256) >= \
+        vs.vs_attn_workspace_size_varlen(3, 4096, 4, 128, 0) + 2 * 12 * 256 * 128 * 2
+
+
 def test_aggregate_host_validation():
     L = vs.lib()
     f = _fake

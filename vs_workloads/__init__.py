@@ -286,3 +286,65 @@ def small_variant(w: Workload, N: int, Hq: int | None = None, Hkv: int | None = 
                     max(1, min(N, int(math.ceil(w.k_v * scale)))),
                     max(1, min(N, int(math.ceil(w.k_s * scale)))), w.tau_v, w.tau_s, w.heads,
                     w.indexer, w.hidden, w.description + f" (scaled to N={N})")
+
+
+@dataclass
+class BatchWorkload:
+    """A batch of independent sequences packed along the token axis
+    (variable-length batched prefill).  Sequence b draws its Q/K/V from seed
+    seed * 100 + b and its scores from the base generator, seed
+    (seed * 100 + b) * 1000 + head; selection per sequence with caps of
+    cap_frac x its length (at least 1)."""
+    name: str
+    lengths: tuple
+    Hq: int
+    Hkv: int
+    d: int
+    rope_base: float
+    seed: int
+    select_mode: str
+    cap_frac: float
+    tau_v: float = 1.0
+    tau_s: float = 1.0
+    description: str = ""
+
+    @property
+    def select_mode_id(self) -> int:
+        return {"topk": 0, "threshold": 1, "maxfrac": 2}[self.select_mode]
+
+    @property
+    def H_sel(self) -> int:
+        return self.Hq
+
+    @property
+    def cu_seqlens(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.lengths)]).astype(np.int32)
+
+    def cap(self, n: int) -> int:
+        return max(1, min(n, int(math.ceil(self.cap_frac * n))))
+
+    def qkv(self):
+        parts = [gen_qkv(self.seed * 100 + b, n, self.Hq, self.Hkv, self.d, self.rope_base)
+                 for b, n in enumerate(self.lengths)]
+        return tuple(np.concatenate([p[t] for p in parts]) for t in range(3))
+
+    def scores(self, b: int):
+        """(logit_v, logit_s) fp32 [H_sel, n] of sequence b."""
+        n = self.lengths[b]
+        lv = np.empty((self.H_sel, n), np.float32)
+        ls = np.empty((self.H_sel, n), np.float32)
+        for h in range(self.H_sel):
+            av, a_s = scores_base(n, (self.seed * 100 + b) * 1000 + h)
+            lv[h], ls[h] = to_logits(av), to_logits(a_s)
+        return lv, ls
+
+
+BATCH_WORKLOADS = {
+    "llama_varlen_mix": BatchWorkload(
+        "llama_varlen_mix",
+        (32768, 24576, 16384, 16384, 12288, 8192, 8192, 4096, 4096, 2048, 2048, 1024, 1024, 512,
+         512, 256, 300),
+        32, 8, 128, 500000.0, 16, "threshold", 0.125, tau_v=0.90, tau_s=0.95,
+        description="17 sequences of 256-32768 tokens (134,700 in all), 32q/8kv, d=128, "
+                    "threshold 0.90/0.95, caps 1/8 of each length"),
+}
