@@ -12,9 +12,12 @@ key) pairs counted exactly from the index sets; ms per layer and the speed-up
 over the library's dense causal kernel on the same inputs are reported too.
 
 Prints ONE JSON line on rank 0.  Multi-GPU: one process per GPU (torchrun);
-every rank runs its own replica of the layer (heads are independent, there is
-no exchange step), timing is the max over ranks, value = all ranks' flops /
-that time ("scaling": "weak").
+by default every rank runs its own replica of the layer (heads are
+independent, there is no exchange step), timing is the max over ranks, value
+= all ranks' flops / that time ("scaling": "weak").  --shard heads splits one
+layer instead: each rank takes Hkv / N KV heads with their query heads and
+index sets (still no exchange step; O stays head-sharded), value = the
+layer's flops summed over ranks / the max rank time ("scaling": "strong").
 
 --impl reference times the fp64 CPU oracle (the only other implementation)
 on bounded row samples of the same workload.
@@ -52,6 +55,8 @@ def parse():
     ap.add_argument("--dense-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="multi-GPU: a replica of the layer per GPU, or the layer's heads split")
     ap.add_argument("--agg-steps", type=int, default=2,
                     help="timed runs of the ground-truth aggregation pass (0: skip)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -108,6 +113,30 @@ def max_over_ranks(values, device=None):
     t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(x) for x in t.tolist()]
+
+
+def sum_over_ranks(values, device=None):
+    """Element-wise sum of a list of floats over all ranks (identity at world 1)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
+
+
+def head_shard(Hq: int, Hkv: int, H_sel: int, world: int, rank: int):
+    """Rank `rank`'s part of a head-sharded layer: whole KV groups, so no rank
+    needs another's K/V.  Returns (q0, q1, kv0, kv1, s0, s1) half-open ranges
+    of query heads, KV heads and index-set heads.  Needs world | Hkv."""
+    if Hkv % world != 0:
+        raise ValueError(f"head sharding needs the GPU count to divide Hkv={Hkv}")
+    kv0, kv1 = rank * Hkv // world, (rank + 1) * Hkv // world
+    G = Hq // Hkv
+    s_per_q = H_sel / Hq
+    q0, q1 = kv0 * G, kv1 * G
+    return q0, q1, kv0, kv1, int(q0 * s_per_q), int(q1 * s_per_q)
 
 
 def whole_job_value(world: int, flops_per_rank: float, ms: float) -> float:
@@ -232,6 +261,16 @@ def run_ours(args, w):
     else:
         lv, ls = w.all_scores()
     gen_s = time.time() - t0
+    sharded = args.shard == "heads" and world > 1
+    H_sel = w.H_sel
+    if sharded:  # this rank's KV groups only
+        q0, q1, kv0, kv1, s0, s1 = head_shard(w.Hq, w.Hkv, w.H_sel, world, rank)
+        Qb = np.ascontiguousarray(Qb[:, q0:q1])
+        Kb = np.ascontiguousarray(Kb[:, kv0:kv1])
+        Vb = np.ascontiguousarray(Vb[:, kv0:kv1])
+        if lv is not None:
+            lv, ls = lv[s0:s1], ls[s0:s1]
+        H_sel = s1 - s0
 
     def to_dev(bits):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -239,7 +278,6 @@ def run_ours(args, w):
     Q, K, V = to_dev(Qb), to_dev(Kb), to_dev(Vb)
     N, Hq, d = Q.shape
     Hkv = K.shape[1]
-    H_sel = w.H_sel
     mode = w.select_mode_id
     if w.indexer:
         W1d, W2d = torch.from_numpy(W1).to(dev), torch.from_numpy(W2).to(dev)
@@ -323,7 +361,9 @@ def run_ours(args, w):
     ms_sel = float(np.mean(sel_ms))
     ms_idx = float(np.mean(idx_ms))
     ms_step, ms_att = max_over_ranks([ms_step, ms_att], dev)
-    value = whole_job_value(world, flops, ms_step)
+    # the job's flops: every replica's, or the shards' sum
+    job_flops = sum_over_ranks([flops], dev)[0] if sharded else world * flops
+    value = job_flops / (ms_step * 1e-3) / 1e12
 
     # dense causal kernel on the same inputs (speed-up denominator)
     ws_dense = vs.workspace(256, dev)
@@ -400,7 +440,7 @@ def run_ours(args, w):
             b.synchronize()
             ts.append(a.elapsed_time(b))
         e2e_ms = max_over_ranks([float(np.min(ts[1:] if len(ts) > 1 else ts))], dev)[0]
-        e2e = {"value": round(whole_job_value(world, flops, e2e_ms), 3), "unit": UNIT,
+        e2e = {"value": round(job_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
@@ -417,11 +457,12 @@ def run_ours(args, w):
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded generators shaped like the pages' workloads)",
-        "config": {"workload": w.name, "N": N, "Hq": Hq, "Hkv": Hkv, "d": d, "H_sel": H_sel,
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded generators shaped like the pages' workloads)",
+        "config": {"workload": w.name, "N": N, "Hq": w.Hq, "Hkv": w.Hkv, "d": d, "H_sel": w.H_sel,
                    "select": w.select_mode, "k_v": w.k_v, "k_s": w.k_s, "tau_v": w.tau_v,
-                   "tau_s": w.tau_s, "indexer": w.indexer, "parallelism": f"replicas x{world}",
+                   "tau_s": w.tau_s, "indexer": w.indexer,
+                   "parallelism": f"heads x{world}" if sharded else f"replicas x{world}",
                    "l2": "inputs exceed L2 (Q/K/V/O resident in HBM) and a 256 MiB buffer is "
                          "written between timed steps, outside the timed windows"},
         "ms_per_layer": round(ms_step, 3), "ms_indexer": round(ms_idx, 3) if w.indexer else None,
