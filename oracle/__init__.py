@@ -57,6 +57,12 @@ def _load():
         lib.or_aggregate.argtypes = [P, P, i32, i32, i32, i32, i32, i64, i64, dbl, P, i32, i64, i64,
                                      P, P]
         lib.or_aggregate.restype = None
+        lib.or_block_select.argtypes = [P, P, i32, i32, i32, i32, i32, i64, i64, dbl, dbl, P, i32,
+                                        P, P]
+        lib.or_block_select.restype = None
+        lib.or_attn_block_rows.argtypes = [P, P, P, i32, i32, i32, i32, i32, i64, i64, dbl, P,
+                                           i32, P, i32, P, P]
+        lib.or_attn_block_rows.restype = None
         _lib = lib
     return _lib
 
@@ -198,3 +204,39 @@ def aggregate(Q, K, heads=None, rows=None, scale=0.0):
     _load().or_aggregate(_ptr(Q), _ptr(K), dtype, N, Hq, Hkv, d, Hq * d, Hkv * d, float(scale),
                          _ptr(heads), heads.size, int(lo), int(hi), _ptr(Av), _ptr(As))
     return Av, As
+
+
+def block_select(Q, K, alpha, heads=None, scale=0.0):
+    """FlashPrefill-style kept key blocks per query block (see vs_oracle.c).
+
+    Returns (mask uint32 [len(heads), T, W], margin float64 [len(heads)])."""
+    dtype = 0 if Q.dtype == np.uint16 else 1
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    Q = np.ascontiguousarray(Q)
+    K = np.ascontiguousarray(K)
+    heads = np.arange(Hq, dtype=np.int32) if heads is None else np.ascontiguousarray(heads, np.int32)
+    T = (N + 127) // 128
+    W = (T + 31) // 32
+    mask = np.zeros((heads.size, T, W), np.uint32)
+    margin = np.zeros(heads.size, np.float64)
+    _load().or_block_select(_ptr(Q), _ptr(K), dtype, N, Hq, Hkv, d, Hq * d, Hkv * d, float(scale),
+                            float(alpha), _ptr(heads), heads.size, _ptr(mask), _ptr(margin))
+    return mask, margin
+
+
+def attn_block_rows(Q, K, V, h, rows, mask, scale=0.0):
+    """Block-sparse causal attention for head h at the given rows; `mask` is
+    [Hq, T, W] as from block_select over all heads.  Returns (O [n, d], lse [n])."""
+    dtype = 0 if Q.dtype == np.uint16 else 1
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    rows = np.ascontiguousarray(rows, np.int64)
+    mask = np.ascontiguousarray(mask, np.uint32)
+    O = np.empty((rows.size, d), np.float64)
+    lse = np.empty(rows.size, np.float64)
+    _load().or_attn_block_rows(_ptr(np.ascontiguousarray(Q)), _ptr(np.ascontiguousarray(K)),
+                               _ptr(np.ascontiguousarray(V)), dtype, N, Hq, Hkv, d, Hq * d, Hkv * d,
+                               float(scale), _ptr(mask), int(h), _ptr(rows), rows.size, _ptr(O),
+                               _ptr(lse))
+    return O, lse

@@ -418,3 +418,124 @@ void or_aggregate(const void* Q, const void* K, int dtype, int N, int Hq, int Hk
     free(s);
   }
 }
+
+/* ------------------------------------------------ FlashPrefill block pattern
+ * FlashPrefill summary page, section 2A (block approximation: a skeleton of
+ * uniformly spaced queries probes the key blocks, with each key block's mean
+ * key as its proxy -- the geometric mean of the block's attention weights,
+ * a monotone proxy of their sum) and section 2B (max-based threshold: for
+ * query block I keep key block J when its score is at least alpha times the
+ * best block's score).  Read here as, with blocks of 128 and B_I the probes
+ * of query block I (rows 128 I + 8 m, m = 0..15, below N):
+ *   kbar_J = mean of the keys of block J (rows below N);
+ *   for J < I:  Score(I, J) = mean over q in B_I of
+ *               softmax_{J' < I}(scale * q . kbar_J')[J];
+ *   keep J < I  iff  Score(I, J) >= alpha * max_{J' < I} Score(I, J');
+ *   the diagonal block J = I is always kept (causal coverage);
+ * all in fp64.  Output: mask [nheads][T][W] words (W = (T + 31) / 32), bit J
+ * of row I set iff block J is kept for query block I.  `margin` receives,
+ * per head, the smallest |Score - alpha max| / (alpha max) over all
+ * decisions, so callers can flag decisions within rounding of the boundary.
+ */
+void or_block_select(const void* Q, const void* K, int dtype, int N, int Hq, int Hkv, int d,
+                     int64_t q_stride_tok, int64_t kv_stride_tok, double scale, double alpha,
+                     const int* heads, int nheads, uint32_t* mask, double* margin) {
+  if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+  const int T = (N + 127) / 128, W = (T + 31) / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int x = 0; x < nheads; ++x) {
+    const int h = heads[x];
+    const int kvh = h / (Hq / Hkv);
+    double* kbar = (double*)calloc((size_t)T * d, sizeof(double));
+    for (int J = 0; J < T; ++J) {
+      int n = 0;
+      for (int64_t j = 128 * (int64_t)J; j < 128 * (int64_t)J + 128 && j < N; ++j, ++n)
+        for (int c = 0; c < d; ++c)
+          kbar[(int64_t)J * d + c] += load_elem(K, dtype, j * kv_stride_tok + (int64_t)kvh * d + c);
+      for (int c = 0; c < d; ++c) kbar[(int64_t)J * d + c] /= (double)n;
+    }
+    double* s = (double*)malloc(sizeof(double) * (size_t)T);
+    double* score = (double*)malloc(sizeof(double) * (size_t)T);
+    double* q = (double*)malloc(sizeof(double) * (size_t)d);
+    double mg = INFINITY;
+    uint32_t* mrow = mask + (int64_t)x * T * W;
+    memset(mrow, 0, sizeof(uint32_t) * (size_t)T * W);
+    for (int I = 0; I < T; ++I) {
+      uint32_t* m = mrow + (int64_t)I * W;
+      m[I >> 5] |= 1u << (I & 31);
+      if (I == 0) continue;
+      for (int J = 0; J < I; ++J) score[J] = 0.0;
+      int np = 0;
+      for (int pm = 0; pm < 16; ++pm) {
+        const int64_t i = 128 * (int64_t)I + 8 * pm;
+        if (i >= N) break;
+        ++np;
+        for (int c = 0; c < d; ++c) q[c] = load_elem(Q, dtype, i * q_stride_tok + (int64_t)h * d + c);
+        double mx = -INFINITY;
+        for (int J = 0; J < I; ++J) {
+          double dot = 0.0;
+          for (int c = 0; c < d; ++c) dot += q[c] * kbar[(int64_t)J * d + c];
+          s[J] = scale * dot;
+          if (s[J] > mx) mx = s[J];
+        }
+        double z = 0.0;
+        for (int J = 0; J < I; ++J) z += exp(s[J] - mx);
+        for (int J = 0; J < I; ++J) score[J] += exp(s[J] - mx) / z;
+      }
+      double best = 0.0;
+      for (int J = 0; J < I; ++J) {
+        score[J] /= (double)np;
+        if (score[J] > best) best = score[J];
+      }
+      const double thr = alpha * best;
+      for (int J = 0; J < I; ++J) {
+        if (score[J] >= thr) m[J >> 5] |= 1u << (J & 31);
+        const double r = fabs(score[J] - thr) / thr;
+        if (r < mg) mg = r;
+      }
+    }
+    margin[x] = mg;
+    free(kbar);
+    free(s);
+    free(score);
+    free(q);
+  }
+}
+
+/* Block-sparse causal attention rows: query i (block I = i / 128) attends
+ * to every key j <= i of every block kept in row I of `mask` (as written by
+ * or_block_select, [Hq][T][W]); softmax and LSE as in or_attn_rows. */
+void or_attn_block_rows(const void* Q, const void* K, const void* V, int dtype, int N, int Hq,
+                        int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok, double scale,
+                        const uint32_t* mask, int h, const int64_t* rows, int nrows, double* O,
+                        double* lse) {
+  or_attn_args a = {0};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.dtype = dtype;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.q_stride_tok = q_stride_tok;
+  a.kv_stride_tok = kv_stride_tok;
+  a.scale = scale > 0.0 ? scale : 1.0 / sqrt((double)d);
+  const int T = (N + 127) / 128, W = (T + 31) / 32;
+#pragma omp parallel
+  {
+    int32_t* keys = (int32_t*)malloc(sizeof(int32_t) * (size_t)N);
+#pragma omp for schedule(dynamic, 16)
+    for (int r = 0; r < nrows; ++r) {
+      const int64_t i = rows[r];
+      const uint32_t* m = mask + ((int64_t)h * T + i / 128) * W;
+      int nk = 0;
+      for (int64_t j = 0; j <= i; ++j) {
+        const int J = (int)(j / 128);
+        if ((m[J >> 5] >> (J & 31)) & 1u) keys[nk++] = (int32_t)j;
+      }
+      softmax_row(&a, h, i, keys, nk, O + (int64_t)r * d, lse + r);
+    }
+    free(keys);
+  }
+}
