@@ -434,8 +434,9 @@ void or_aggregate(const void* Q, const void* K, int dtype, int N, int Hq, int Hk
  *   the diagonal block J = I is always kept (causal coverage);
  * all in fp64.  Output: mask [nheads][T][W] words (W = (T + 31) / 32), bit J
  * of row I set iff block J is kept for query block I.  `margin` receives,
- * per head, the smallest |Score - alpha max| / (alpha max) over all
- * decisions, so callers can flag decisions within rounding of the boundary.
+ * per head, the smallest |Score - alpha max| / (alpha max) over the
+ * decisions other than the best block's (kept for any alpha <= 1), so callers
+ * can flag decisions within rounding of the boundary.
  */
 void or_block_select(const void* Q, const void* K, int dtype, int N, int Hq, int Hkv, int d,
                      int64_t q_stride_tok, int64_t kv_stride_tok, double scale, double alpha,
@@ -490,6 +491,7 @@ void or_block_select(const void* Q, const void* K, int dtype, int N, int Hq, int
       const double thr = alpha * best;
       for (int J = 0; J < I; ++J) {
         if (score[J] >= thr) m[J >> 5] |= 1u << (J & 31);
+        if (score[J] == best) continue;  /* the best block is kept for any alpha <= 1 */
         const double r = fabs(score[J] - thr) / thr;
         if (r < mg) mg = r;
       }
