@@ -208,6 +208,48 @@ vs_status vs_dense_attn_fwd_varlen(const void* Q, const void* K, const void* V, 
                                    void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * vs_block_select -- FlashPrefill's block pattern discovery (FlashPrefill
+ * summary page, section 2A: a skeleton of uniformly spaced queries probes
+ * every key block through the block's mean key, a proxy that is monotone in
+ * the block's total attention weight; section 2B: keep key block J for query
+ * block I when its score is at least alpha times the best block's -- no
+ * sort, no cumulative sum).  Read as, with 128-row blocks and the probes of
+ * block I at rows 128 I + 8 m (m = 0..15, below N):
+ *     Score(I, J) = mean over probes q of softmax_{J' < I}(scale q . kbar_J')[J],
+ *     J < I kept iff Score(I, J) >= alpha * max_J' Score(I, J'),
+ * the diagonal block J = I always kept; computed in fp64.
+ *   Q [N, Hq, d], K [N, Hkv, d] (VS_BF16 or VS_FP32; strides as for the
+ *            attention calls).  1 <= N <= 2^18.  0 < alpha <= 1.
+ *   mask     uint32 [Hq][T][W] output (device), T = ceil(N / 128),
+ *            W = ceil(T / 32): bit J of row (h, I) set iff block J is kept.
+ *   ws       at least vs_block_select_workspace_size(N, Hkv, d) bytes,
+ *            256-byte aligned (status word, then the fp64 block means).
+ */
+size_t vs_block_select_workspace_size(int N, int Hkv, int d);
+vs_status vs_block_select(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
+                          int d, int64_t q_stride_tok, int64_t kv_stride_tok, float softmax_scale,
+                          double alpha, uint32_t* mask, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/*
+ * vs_block_sparse_attn_fwd -- causal attention over kept key blocks
+ * (FlashPrefill summary page, section 3: a block-sparse kernel that jumps
+ * directly to the next kept block by index).  Query i (block I = i / 128)
+ * attends to every key j <= i of every block J kept in row (h, I) of
+ * `block_mask` (the layout vs_block_select writes; bits J > I are ignored).
+ * O and lse as for vs_sparse_attn_fwd; a row with no kept key gets O = 0 and
+ * LSE = -inf.  VS_BF16 only; 1 <= N <= 2^18.
+ *   ws       at least vs_block_attn_workspace_size(N, Hq) bytes, 256-byte
+ *            aligned (status word and the per-pair block lists).
+ */
+size_t vs_block_attn_workspace_size(int N, int Hq);
+vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                   int N, int Hq, int Hkv, int d, int64_t q_stride_tok,
+                                   int64_t kv_stride_tok, float softmax_scale,
+                                   const uint32_t* block_mask, void* O, float* lse, void* ws,
+                                   size_t ws_bytes, cudaStream_t stream);
+
+/*
  * vs_sparse_attn_fwd_static_scratch -- vs_sparse_attn_fwd without a
  * caller-provided workspace.  The summary pages have no counterpart to this
  * call; it exists for callers that cannot allocate device memory: plain-C

@@ -42,7 +42,8 @@ EXPORTS = (
     "vs_attn_workspace_size", "vs_sparse_attn_fwd", "vs_dense_attn_fwd", "vs_read_device_status",
     "vs_selftest_wait_timeout", "vs_sparse_attn_fwd_static_scratch", "vs_attn_workspace_size_ld",
     "vs_attn_aggregate", "vs_attn_workspace_size_varlen", "vs_sparse_attn_fwd_varlen",
-    "vs_dense_attn_fwd_varlen",
+    "vs_dense_attn_fwd_varlen", "vs_block_select_workspace_size", "vs_block_select",
+    "vs_block_attn_workspace_size", "vs_block_sparse_attn_fwd",
 )
 
 
@@ -95,6 +96,15 @@ def lib() -> ctypes.CDLL:
         L.vs_dense_attn_fwd_varlen.argtypes = [P, P, P, I, I, I, P, I, I, I, I, I64, I64, F, P, P,
                                                P, Z, P]
         L.vs_dense_attn_fwd_varlen.restype = I
+        L.vs_block_select_workspace_size.argtypes = [I, I, I]
+        L.vs_block_select_workspace_size.restype = Z
+        L.vs_block_select.argtypes = [P, P, I, I, I, I, I, I64, I64, F, D, P, P, Z, P]
+        L.vs_block_select.restype = I
+        L.vs_block_attn_workspace_size.argtypes = [I, I]
+        L.vs_block_attn_workspace_size.restype = Z
+        L.vs_block_sparse_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, P, P, P, P, Z,
+                                               P]
+        L.vs_block_sparse_attn_fwd.restype = I
         L.vs_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
         L.vs_read_device_status.restype = I
         L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
@@ -238,6 +248,46 @@ def vs_dense_attn_fwd_varlen(Q, K, V, cu_seqlens, max_seqlen, O, lse, ws, softma
         _ptr(Q), _ptr(K), _ptr(V), _dtype(Q), T, B, _ptr(cu_seqlens), int(max_seqlen), Hq, Hkv, d,
         Q.stride(0), K.stride(0), float(softmax_scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
         _stream(stream)), "vs_dense_attn_fwd_varlen")
+
+
+def vs_block_select_workspace_size(N: int, Hkv: int, d: int) -> int:
+    return int(lib().vs_block_select_workspace_size(N, Hkv, d))
+
+
+def vs_block_attn_workspace_size(N: int, Hq: int) -> int:
+    return int(lib().vs_block_attn_workspace_size(N, Hq))
+
+
+def vs_block_select(Q, K, alpha, mask, ws, softmax_scale=0.0, stream=None):
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    _check(lib().vs_block_select(_ptr(Q), _ptr(K), _dtype(Q), N, Hq, Hkv, d, Q.stride(0),
+                                 K.stride(0), float(softmax_scale), float(alpha), _ptr(mask),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "vs_block_select")
+
+
+def vs_block_sparse_attn_fwd(Q, K, V, mask, O, lse, ws, softmax_scale=0.0, stream=None):
+    N, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    _check(lib().vs_block_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype(Q), N, Hq, Hkv, d,
+                                          Q.stride(0), K.stride(0), float(softmax_scale),
+                                          _ptr(mask), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "vs_block_sparse_attn_fwd")
+
+
+def block_prefill(Q, K, V, alpha, stream=None):
+    """FlashPrefill-style pattern discovery then block-sparse attention:
+    returns (O, lse, mask)."""
+    N, Hq, d = Q.shape
+    T = (N + 127) // 128
+    mask = torch.empty((Hq, T, (T + 31) // 32), dtype=torch.int32, device=Q.device)
+    ws = workspace(max(vs_block_select_workspace_size(N, K.shape[1], d),
+                       vs_block_attn_workspace_size(N, Hq)), Q.device)
+    vs_block_select(Q, K, alpha, mask, ws, stream=stream)
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, N), dtype=torch.float32, device=Q.device)
+    vs_block_sparse_attn_fwd(Q, K, V, mask, O, lse, ws, stream=stream)
+    return O, lse, mask
 
 
 def vs_read_device_status(ws, stream=None) -> tuple[int, int]:

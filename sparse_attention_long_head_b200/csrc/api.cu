@@ -188,6 +188,7 @@ static vs_status attn_impl(const void* Q, const void* K, const void* V, vs_dtype
   a.kv_stride = kv_stride_tok;
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
   a.sparse = sparse;
+  a.block_mask = nullptr;
   a.v_idx = v_idx;
   a.v_ld = v_ld;
   a.v_cnt = v_cnt;
@@ -297,6 +298,88 @@ vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N,
   if (cudaMemsetAsync(A_s, 0, sizeof(float) * (size_t)Hq * (size_t)N, stream) != cudaSuccess)
     return VS_ERR_CUDA;
   return launch_aggregate(a) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
+size_t vs_block_select_workspace_size(int N, int Hkv, int d) {
+  if (N < 1 || Hkv < 1 || d < 1) return kStatusBytes;
+  return block_select_ws_bytes(N, Hkv, d);
+}
+
+vs_status vs_block_select(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
+                          int d, int64_t q_stride_tok, int64_t kv_stride_tok, float softmax_scale,
+                          double alpha, uint32_t* mask, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  if (!mask) return VS_ERR_INVALID_ARG;
+  vs_status st = check_attn_common(Q, K, K, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
+                                   softmax_scale, mask);
+  if (st != VS_OK) return st;
+  if (!(alpha > 0.0 && alpha <= 1.0)) return VS_ERR_INVALID_ARG;
+  if (N > (1 << 18)) return VS_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < block_select_ws_bytes(N, Hkv, d) || !aligned(ws, 256))
+    return VS_ERR_WORKSPACE;
+  BlockSelectArgs a;
+  a.Q = Q;
+  a.K = K;
+  a.dtype = dtype;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.q_stride = q_stride_tok;
+  a.kv_stride = kv_stride_tok;
+  a.scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)d);
+  a.alpha = alpha;
+  a.mask = mask;
+  a.ws = ws;
+  a.stream = stream;
+  if (cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  return launch_block_select(a) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
+size_t vs_block_attn_workspace_size(int N, int Hq) {
+  if (N < 1 || Hq < 1) return kStatusBytes;
+  return BlockPlanLayout::make(N, Hq).total;
+}
+
+vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                   int N, int Hq, int Hkv, int d, int64_t q_stride_tok,
+                                   int64_t kv_stride_tok, float softmax_scale,
+                                   const uint32_t* block_mask, void* O, float* lse, void* ws,
+                                   size_t ws_bytes, cudaStream_t stream) {
+  if (!block_mask) return VS_ERR_INVALID_ARG;
+  vs_status st = check_attn_common(Q, K, V, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
+                                   softmax_scale, O);
+  if (st != VS_OK) return st;
+  if (dtype != VS_BF16 || N > (1 << 18)) return VS_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < BlockPlanLayout::make(N, Hq).total || !aligned(ws, 256))
+    return VS_ERR_WORKSPACE;
+  AttnArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.O = O;
+  a.lse = lse;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.H_sel = 1;
+  a.B = 1;
+  a.total = N;
+  a.cu_seqlens = nullptr;
+  a.q_stride = q_stride_tok;
+  a.kv_stride = kv_stride_tok;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+  a.sparse = false;
+  a.block_mask = block_mask;
+  a.ws = ws;
+  a.status = static_cast<int*>(ws);
+  a.stream = stream;
+  a.pack_vrows = 0;
+  const PlanLayout L = PlanLayout::make(N, 1);  // tile and pair counts
+  if (cudaMemsetAsync(a.status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  if (launch_block_plan(a) != cudaSuccess) return VS_ERR_CUDA;
+  return launch_attn_tc(a, L) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
 }
 
 vs_status vs_read_device_status(const void* ws, cudaStream_t stream, int* flags) {

@@ -257,13 +257,69 @@ cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------ block plan
+
+// For each (head h, pair p) of query blocks I = 2p, 2p + 1: the ascending
+// union of the key blocks kept for either (J <= I each), with bit 30 / 31
+// marking the blocks kept for the first / second.  One warp per unit; the
+// rows have at most 64 words (T <= 2048).
+__global__ void __launch_bounds__(32) block_plan_kernel(const uint32_t* mask, int T, int P,
+                                                        int32_t* bcnt, uint32_t* blist) {
+  const int p = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
+  const int W = (T + 31) / 32;
+  const int IA = 2 * p, IB = 2 * p + 1;
+  const uint32_t* ra = mask + ((int64_t)h * T + IA) * W;
+  const uint32_t* rb = IB < T ? mask + ((int64_t)h * T + IB) * W : nullptr;
+  uint32_t* out = blist + (int64_t)h * P * (P + 1) + (int64_t)p * (p + 1);
+  auto upto = [](int w, int last) -> uint32_t {  // bits of word w at positions <= last
+    const int k = last - 32 * w;
+    return k < 0 ? 0u : (k >= 31 ? 0xffffffffu : ((2u << k) - 1u));
+  };
+  int base = 0;
+  for (int w0 = 0; w0 < W; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t a = 0u, b = 0u;
+    if (w < W) {
+      a = ra[w] & upto(w, IA);
+      b = rb ? rb[w] & upto(w, min(IB, T - 1)) : 0u;
+    }
+    const uint32_t u = a | b;
+    const int c = __popc(u);
+    int incl = c;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = base + incl - c;
+    uint32_t x = u;
+    while (x) {
+      const int bit = __ffs(x) - 1;
+      x &= x - 1;
+      const uint32_t J = 32u * w + bit;
+      out[pos++] = J | (((a >> bit) & 1u) << 30) | (((b >> bit) & 1u) << 31);
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) bcnt[(int64_t)h * P + p] = base;
+}
+
+cudaError_t launch_block_plan(const AttnArgs& a) {
+  const BlockPlanLayout B = BlockPlanLayout::make(a.N, a.Hq);
+  int32_t* bcnt = reinterpret_cast<int32_t*>(static_cast<char*>(a.ws) + B.off_cnt);
+  uint32_t* blist = reinterpret_cast<uint32_t*>(static_cast<char*>(a.ws) + B.off_list);
+  block_plan_kernel<<<dim3(B.P, a.Hq), 32, 0, a.stream>>>(a.block_mask, B.T, B.P, bcnt, blist);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------- attention
 
 constexpr int kAttnThreads = 320;
 constexpr int kWarpMMA = 8;
 constexpr int kWarpLoad = 9;
 
-enum : int { kModeDense = 0, kModeDenseVS = 1, kModeSplit = 2 };
+enum : int { kModeDense = 0, kModeDenseVS = 1, kModeSplit = 2, kModeBlock = 3 };
+// Kernel instantiations: dense causal, vertical-slash sparse, block sparse.
+enum : int { kAttnDense = 0, kAttnVS = 1, kAttnBlock = 2 };
 enum : int { kItemTile = 0, kItemVChunk = 1 };
 
 template <int D>
@@ -291,6 +347,11 @@ struct AttnParams {
   PlanLayout L;
   PlanPtrs pp;
   int64_t pack_vrows;  // 0: gather vertical rows; else packed tiles (tmKg/tmVg map them)
+  // block sparse: per (head, pair) the count and, at h P (P + 1) + p (p + 1),
+  // the ascending kept key blocks of both query blocks (bit 30: kept for the
+  // first, bit 31: for the second)
+  const int32_t* bcnt;
+  const uint32_t* blist;
 };
 
 struct UnitInfo {
@@ -305,7 +366,7 @@ __device__ __forceinline__ int64_t unit_tok0(const AttnParams& P, const UnitInfo
   return P.cu ? (int64_t)__ldg(P.cu + ui.b) : 0;
 }
 
-template <bool SPARSE>
+template <int MODE>
 __device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
   // Units grouped by KV head (so CTAs running at the same time stream the same
   // K/V and share it in L2), heaviest (largest p) first within a group, the G
@@ -334,9 +395,15 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
     ui.n = 0;
     return ui;
   }
-  if (!SPARSE) {
+  if (MODE == kAttnDense) {
     ui.mode = kModeDense;
     ui.n = n_dense;
+    return ui;
+  }
+  if (MODE == kAttnBlock) {
+    ui.mode = kModeBlock;
+    ui.n = P.bcnt[(int64_t)ui.h * P.P + ui.p];
+    ui.d1start = ui.h * P.P * (P.P + 1) + ui.p * (ui.p + 1);
     return ui;
   }
   const int32_t* d1pref = P.pp.d1pref + (int64_t)ui.hs * P.L.d1pref_len;
@@ -360,12 +427,19 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
 
 struct Item {
   int kind;
-  int b;  // key block (tile) or chunk index (vertical chunk)
+  int b;      // key block (tile) or chunk index (vertical chunk)
+  int flags;  // block sparse: bit s set iff the block is kept for sub-tile s
 };
 
 __device__ __forceinline__ Item unit_item(const AttnParams& P, const UnitInfo& ui, int k) {
   Item it;
-  if (ui.mode != kModeSplit) {
+  it.flags = 3;
+  if (ui.mode == kModeBlock) {
+    const uint32_t e = P.blist[(int64_t)ui.d1start + k];
+    it.kind = kItemTile;
+    it.b = (int)(e & 0xFFFFu);
+    it.flags = (int)(e >> 30);
+  } else if (ui.mode != kModeSplit) {
     it.kind = kItemTile;
     it.b = k;
   } else if (k < ui.nvc) {
@@ -385,7 +459,7 @@ __device__ __forceinline__ uint32_t prefix_word(int n, int lo) {
 }
 
 // 128-bit keep-mask of row i for one item; returns false if every key is kept.
-template <bool SPARSE>
+template <int MODE>
 __device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& ui, const Item& it,
                                           int i, int t_sub, uint32_t (&w)[4]) {
   if (it.kind == kItemVChunk) {
@@ -409,7 +483,12 @@ __device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& u
   const int b = it.b;
   // causal part for the keys of block b: keep c <= i - 128 b
   const bool below = b < t_sub;  // whole block in the past of every row of the sub-tile
-  if (!SPARSE || ui.mode == kModeDense) {
+  if (MODE == kAttnBlock && !((it.flags >> (t_sub - 2 * ui.p)) & 1)) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = 0u;  // not kept for this sub-tile's query block
+    return true;
+  }
+  if (MODE != kAttnVS || ui.mode == kModeDense) {
     if (below) return false;
     const int n = i - 128 * b + 1;
 #pragma unroll
@@ -503,7 +582,7 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&sr)[4][32], const uint
   ls = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-template <int D, bool SPARSE>
+template <int D, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKg,
@@ -549,7 +628,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    if (SPARSE) {
+    if (MODE == kAttnVS) {
       tma_prefetch_desc(&tmKg);
       tma_prefetch_desc(&tmVg);
     }
@@ -563,7 +642,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tslot;
   const WaitCtx wc{P.wait_limit_ns, P.status, abort_flag};
-  if (!SPARSE && P.cu && blockIdx.x == 0 && tid == 0) {
+  if (MODE == kAttnDense && P.cu && blockIdx.x == 0 && tid == 0) {
     // the sparse path's plan kernel checks the offsets; here the first CTA does
     for (int b = 0; b < P.B; ++b) {
       int64_t t0;
@@ -582,7 +661,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t scnt = 0, ucount = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
-      const UnitInfo ui = unit_info<SPARSE>(P, u);
+      const UnitInfo ui = unit_info<MODE>(P, u);
       const int i = 256 * ui.p + 128 * sub + r;
       const int im = max(0, min(i, ui.Nb - 1));
       const int t_sub = 2 * ui.p + sub;
@@ -605,7 +684,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int k = 0; k < ui.n; ++k) {
         const Item it = unit_item(P, ui, k);
         uint32_t mw[4];
-        const bool masked = item_mask<SPARSE>(P, ui, it, im, t_sub, mw);
+        const bool masked = item_mask<MODE>(P, ui, it, im, t_sub, mw);
         if (!mbar_wait(bar(B_SFULL + sub), scnt & 1, wc)) { ok = false; break; }
         ++scnt;
         tc_fence_after();
@@ -726,7 +805,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kk = 1; kk < 8; ++kk) mma_ts(d, a + kk * 8, bd + ((kk * 2048) >> 4), idesc_pv, 1u);
       };
       for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
-        const UnitInfo ui = unit_info<SPARSE>(P, u);
+        const UnitInfo ui = unit_info<MODE>(P, u);
         if (ui.n == 0) continue;
         if (!mbar_wait(bar(B_QFULL), ucount & 1, wc)) { ok = false; break; }
         uint32_t kslot = seq % S;
@@ -781,7 +860,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     bool ok = true;
     const int nsub64 = D / 64;
     for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
-      const UnitInfo ui = unit_info<SPARSE>(P, u);
+      const UnitInfo ui = unit_info<MODE>(P, u);
       if (ui.n == 0) continue;
       if (ucount > 0 && !mbar_wait(bar(B_QEMPTY), (ucount - 1) & 1, wc)) { ok = false; break; }
       const int64_t tok0 = unit_tok0(P, ui);
@@ -876,8 +955,9 @@ static void encode_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int6
   if (r != CUDA_SUCCESS) *rc = r;
 }
 
-template <int D, bool SPARSE>
+template <int D, int MODE>
 static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
+  constexpr bool SPARSE = MODE == kAttnVS;
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap mQ, mK, mV, mKg, mVg;
@@ -914,7 +994,14 @@ static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
   P.L = L;
   P.pp = plan_ptrs(L, a.ws);
   P.pack_vrows = SPARSE ? a.pack_vrows : 0;
-  auto kern = attn_tc_kernel<D, SPARSE>;
+  P.bcnt = nullptr;
+  P.blist = nullptr;
+  if (MODE == kAttnBlock) {
+    const BlockPlanLayout B = BlockPlanLayout::make(a.N, a.Hq);
+    P.bcnt = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.ws) + B.off_cnt);
+    P.blist = reinterpret_cast<const uint32_t*>(static_cast<const char*>(a.ws) + B.off_list);
+  }
+  auto kern = attn_tc_kernel<D, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg<D>::kSmem);
   if (e != cudaSuccess) return e;
@@ -924,8 +1011,15 @@ static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, const PlanLayout& L) {
-  if (a.d == 128) return a.sparse ? launch_tc_impl<128, true>(a, L) : launch_tc_impl<128, false>(a, L);
-  if (a.d == 64) return a.sparse ? launch_tc_impl<64, true>(a, L) : launch_tc_impl<64, false>(a, L);
+  if (a.block_mask) {
+    if (a.d == 128) return launch_tc_impl<128, kAttnBlock>(a, L);
+    if (a.d == 64) return launch_tc_impl<64, kAttnBlock>(a, L);
+    return cudaErrorInvalidValue;
+  }
+  if (a.d == 128)
+    return a.sparse ? launch_tc_impl<128, kAttnVS>(a, L) : launch_tc_impl<128, kAttnDense>(a, L);
+  if (a.d == 64)
+    return a.sparse ? launch_tc_impl<64, kAttnVS>(a, L) : launch_tc_impl<64, kAttnDense>(a, L);
   return cudaErrorInvalidValue;
 }
 

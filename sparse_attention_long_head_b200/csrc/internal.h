@@ -139,6 +139,23 @@ __host__ __device__ inline bool seq_range(const int32_t* cu, int64_t total, int 
   return true;
 }
 
+// Block-sparse plan in the workspace (after the status header): per (head,
+// pair of query blocks) a count, and the kept key blocks of the pair at
+// h P (P + 1) + p (p + 1) (at most 2p + 2 of them).
+struct BlockPlanLayout {
+  int T = 0, P = 0;
+  size_t off_cnt = 0, off_list = 0, total = 0;
+  __host__ __device__ static BlockPlanLayout make(int N, int Hq) {
+    BlockPlanLayout B;
+    B.T = (N + 127) / 128;
+    B.P = (B.T + 1) / 2;
+    B.off_cnt = 256;
+    B.off_list = B.off_cnt + (sizeof(int32_t) * (size_t)Hq * B.P + 255) / 256 * 256;
+    B.total = B.off_list + sizeof(uint32_t) * (size_t)Hq * B.P * (B.P + 1);
+    return B;
+  }
+};
+
 // Common attention launch description.  A batch of B sequences packed along
 // the token axis (cu_seqlens, device, B + 1 offsets; null for one sequence)
 // has plan slots b * H_sel + hs, each laid out for N = the longest sequence.
@@ -155,6 +172,7 @@ struct AttnArgs {
   int64_t q_stride, kv_stride;
   float scale;
   bool sparse;
+  const uint32_t* block_mask;  // block sparse: kept key blocks [Hq][T][W] (else null)
   const int32_t* v_idx;
   int64_t v_ld;
   const int32_t* v_cnt;
@@ -184,9 +202,24 @@ struct AggArgs {
   cudaStream_t stream;
 };
 
+// FlashPrefill-style block pattern discovery (blocks.cu).
+struct BlockSelectArgs {
+  const void* Q;
+  const void* K;
+  int dtype, N, Hq, Hkv, d;
+  int64_t q_stride, kv_stride;
+  double scale, alpha;
+  uint32_t* mask;  // [Hq][T][W]
+  void* ws;        // status word, then the block means
+  cudaStream_t stream;
+};
+size_t block_select_ws_bytes(int N, int Hkv, int d);
+cudaError_t launch_block_select(const BlockSelectArgs& a);
+
 // Launchers (return a CUDA error; argument checks are done by the caller).
 cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L);
+cudaError_t launch_block_plan(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_attn_fp32(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,

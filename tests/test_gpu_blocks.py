@@ -1,0 +1,118 @@
+"""FlashPrefill-style block pattern discovery and block-sparse attention on
+the GPU vs the oracle (FlashPrefill summary page, sections 2A, 2B and 3).
+
+Selection: bit-exact kept-block masks on the same inputs (both sides decide
+in fp64; a decision within 1e-9 of its threshold would be a tie zone, and the
+seeds give none).  Attention: bf16 tolerances as for the other kernels, on
+the oracle's own masks."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_long_head_b200 as vs
+from vs_testutil import bf16_to_dev, compare_rows, dev_to_f64
+from vs_workloads import gen_qkv, plant_block_structure
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_mask(Q, K, alpha):
+    N, Hq, d = Q.shape
+    T = (N + 127) // 128
+    mask = torch.zeros((Hq, T, (T + 31) // 32), dtype=torch.int32, device="cuda")
+    ws = vs.workspace(vs.vs_block_select_workspace_size(N, K.shape[1], d))
+    vs.vs_block_select(Q, K, alpha, mask, ws)
+    rc, flags = vs.vs_read_device_status(ws)
+    assert rc == vs.VS_OK and flags == 0
+    return mask.cpu().numpy().view(np.uint32)
+
+
+@pytest.mark.parametrize("N,d,Hq,Hkv,alpha", [(128, 128, 2, 1, 0.5), (1000, 128, 4, 2, 0.2),
+                                              (3000, 64, 4, 1, 0.05), (4097, 128, 2, 2, 0.6),
+                                              (2500, 128, 8, 2, 1.0)])
+def test_block_select_against_oracle(N, d, Hq, Hkv, alpha, cuda_device):
+    Qb, Kb, _ = gen_qkv(N + 3, N, Hq, Hkv, d, 10000.0)
+    Qb, Kb = plant_block_structure(Qb, Kb, seed=N)
+    ref, margin = oracle.block_select(Qb, Kb, alpha)
+    assert (margin > 1e-9).all(), margin
+    got = _gpu_mask(bf16_to_dev(Qb), bf16_to_dev(Kb), alpha)
+    assert np.array_equal(got, ref)
+
+
+def _gpu_block_attn(Qb, Kb, Vb, mask):
+    Q, K, V = (bf16_to_dev(x) for x in (Qb, Kb, Vb))
+    N, Hq, d = Q.shape
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, N), dtype=torch.float32, device="cuda")
+    ws = vs.workspace(vs.vs_block_attn_workspace_size(N, Hq))
+    vs.vs_block_sparse_attn_fwd(Q, K, V, torch.from_numpy(mask.view(np.int32)).cuda(), O, lse, ws)
+    rc, flags = vs.vs_read_device_status(ws)
+    assert rc == vs.VS_OK and flags == 0
+    return O, lse
+
+
+@pytest.mark.parametrize("N,d,Hq,Hkv,alpha", [(1000, 128, 4, 2, 0.2), (129, 64, 2, 1, 0.5),
+                                              (3000, 128, 2, 1, 0.05), (2049, 64, 4, 4, 0.9)])
+def test_block_attention_against_oracle(N, d, Hq, Hkv, alpha, cuda_device):
+    Qb, Kb, Vb = gen_qkv(N + 7, N, Hq, Hkv, d, 10000.0)
+    Qb, Kb = plant_block_structure(Qb, Kb, seed=N + 1)
+    mask, _ = oracle.block_select(Qb, Kb, alpha)
+    O, lse = _gpu_block_attn(Qb, Kb, Vb, mask)
+    Od = dev_to_f64(O)
+    lsed = lse.cpu().numpy().astype(np.float64)
+    rows = np.arange(N)
+    for h in range(Hq):
+        Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, rows, mask)
+        compare_rows(Od[:, h], Or, lsed[h], lr, what=f"block N={N} head {h}")
+
+
+def test_all_blocks_kept_equals_dense_kernel_bitwise(cuda_device):
+    N, Hq = 1500, 4
+    Qb, Kb, Vb = gen_qkv(11, N, Hq, 2, 128, 10000.0)
+    T = (N + 127) // 128
+    W = (T + 31) // 32
+    mask = np.zeros((Hq, T, W), np.uint32)
+    for I in range(T):
+        for J in range(I + 1):
+            mask[:, I, J >> 5] |= np.uint32(1 << (J & 31))
+    O, lse = _gpu_block_attn(Qb, Kb, Vb, mask)
+    Od, lsed = vs.dense_attention(*(bf16_to_dev(x) for x in (Qb, Kb, Vb)))
+    assert torch.equal(O, Od) and torch.equal(lse, lsed)
+
+
+def test_unkept_rows_and_ignored_upper_bits(cuda_device):
+    # row I keeps nothing (not even its diagonal) -> O = 0, LSE = -inf there;
+    # bits above the diagonal are ignored
+    N, Hq = 700, 2
+    Qb, Kb, Vb = gen_qkv(12, N, Hq, 1, 128, 10000.0)
+    T = (N + 127) // 128
+    mask = np.full((Hq, T, 1), 0xFFFFFFFF, np.uint32)
+    mask[0, 2, 0] = 0
+    O, lse = _gpu_block_attn(Qb, Kb, Vb, mask)
+    clean = mask.copy()
+    for I in range(T):
+        clean[:, I, 0] &= np.uint32((1 << (I + 1)) - 1)
+    Od = dev_to_f64(O)
+    lsed = lse.cpu().numpy().astype(np.float64)
+    for h in range(Hq):
+        Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, np.arange(N), clean)
+        compare_rows(Od[:, h], Or, lsed[h], lr, what=f"head {h}")
+    assert np.all(Od[256:384, 0] == 0) and np.all(np.isneginf(lsed[0, 256:384]))
+
+
+def test_block_prefill_pipeline(cuda_device):
+    N, Hq, Hkv, d, alpha = 4000, 4, 2, 128, 0.1
+    Qb, Kb, Vb = gen_qkv(13, N, Hq, Hkv, d, 500000.0)
+    Qb, Kb = plant_block_structure(Qb, Kb, seed=3)
+    O, lse, mask = vs.block_prefill(*(bf16_to_dev(x) for x in (Qb, Kb, Vb)), alpha)
+    ref, margin = oracle.block_select(Qb, Kb, alpha)
+    assert (margin > 1e-9).all()
+    assert np.array_equal(mask.cpu().numpy().view(np.uint32), ref)
+    Od = dev_to_f64(O)
+    lsed = lse.cpu().numpy().astype(np.float64)
+    rows = np.unique(np.concatenate([np.arange(0, 300), np.arange(N - 300, N),
+                                     np.random.default_rng(0).integers(0, N, 300)]))
+    for h in range(Hq):
+        Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, rows, ref)
+        compare_rows(Od[rows, h], Or, lsed[h, rows], lr, what=f"pipeline head {h}")

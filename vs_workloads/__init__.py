@@ -348,3 +348,36 @@ BATCH_WORKLOADS = {
         description="17 sequences of 256-32768 tokens (134,700 in all), 32q/8kv, d=128, "
                     "threshold 0.90/0.95, caps 1/8 of each length"),
 }
+
+
+def plant_block_structure(Qb: np.ndarray, Kb: np.ndarray, seed: int, sinks: int = 3,
+                          strength: float = 5.8, local: float = 4.8, period: float = 2048.0):
+    """Block-level attention structure on top of bf16 Q/K bits (returns new
+    bits): per KV head a random unit direction u is added to every query of
+    its group (x strength) and to the keys of block 0 and `sinks` random
+    blocks (x strength), so those blocks act as sinks (a logit bump of about
+    strength^2 / sqrt(d)); and a slow rotation in two further directions,
+    local * (cos(w t) e1 + sin(w t) e2) with w = 2 pi / period, is added to
+    queries and keys at position t, so nearby blocks score higher (a bump of
+    about local^2 cos(w (i - j)) / sqrt(d)).  The result is rounded to bf16
+    once (round to nearest even)."""
+    N, Hq, d = Qb.shape
+    Hkv = Kb.shape[1]
+    G = Hq // Hkv
+    T = (N + 127) // 128
+    rng = np.random.default_rng([seed, 7])
+    q = bf16_bits_to_f32(Qb).astype(np.float64)
+    k = bf16_bits_to_f32(Kb).astype(np.float64)
+    t = np.arange(N, dtype=np.float64)
+    w = 2.0 * np.pi / period
+    rot = np.stack([np.cos(w * t), np.sin(w * t)], 1)  # [N, 2]
+    for g in range(Hkv):
+        basis, _ = np.linalg.qr(rng.standard_normal((d, 3)))
+        u, e = basis[:, 0], basis[:, 1:3]
+        blocks = np.unique(np.concatenate([[0], rng.integers(0, T, sinks)]))
+        for J in blocks:
+            k[128 * J:128 * J + 128, g] += strength * u
+        k[:, g] += local * rot @ e.T
+        for h in range(g * G, (g + 1) * G):
+            q[:, h] += strength * u + local * rot @ e.T
+    return f64_to_bf16_bits(q), f64_to_bf16_bits(k)
