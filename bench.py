@@ -37,7 +37,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from vs_workloads import BATCH_WORKLOADS, WORKLOADS  # noqa: E402
+from vs_workloads import BATCH_WORKLOADS, BLOCK_WORKLOADS, WORKLOADS  # noqa: E402
 
 METRIC = "VS-sparse prefill ms/layer & effective TFLOP/s at 128K; speedup vs dense"
 UNIT = "TFLOP/s"
@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama_128k",
-                    choices=sorted(WORKLOADS) + sorted(BATCH_WORKLOADS))
+                    choices=sorted(WORKLOADS) + sorted(BATCH_WORKLOADS) + sorted(BLOCK_WORKLOADS))
     ap.add_argument("--dense-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -879,8 +879,241 @@ def run_batch(args, w):
         print(json.dumps(out), flush=True)
 
 
+def block_pairs(mask: np.ndarray, N: int) -> int:
+    """Causal (query, key) pairs inside the kept blocks of a [H, T, W] mask."""
+    H, T, _ = mask.shape
+    bits = np.unpackbits(np.ascontiguousarray(mask).view(np.uint8), bitorder="little")
+    bits = bits.reshape(H, T, -1)[:, :, :T].astype(bool)
+    rows = np.minimum(N - 128 * np.arange(T), 128)          # query rows of block I
+    cols = np.minimum(N - 128 * np.arange(T), 128)          # keys of block J
+    total = 0
+    for I in range(T):
+        kept = bits[:, I, :I].sum()
+        total += int(kept) * 128 * int(rows[I]) if I else 0   # full past blocks (128 keys each)
+        diag = int(bits[:, I, I].sum())
+        total += diag * int(rows[I]) * (int(rows[I]) + 1) // 2
+    return total
+
+
+def run_blocks(args, w):
+    """FlashPrefill-style step: block pattern discovery then block-sparse
+    attention; value = 4 d x (causal pairs in the kept blocks) / step time."""
+    import torch
+    import torch.distributed as dist
+    import sparse_attention_long_head_b200 as vs
+
+    world, rank, local_rank = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    t0 = time.time()
+    Qb, Kb, Vb = w.qkv()
+    gen_s = time.time() - t0
+    to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    Q, K, V = to_dev(Qb), to_dev(Kb), to_dev(Vb)
+    N, Hq, d = Q.shape
+    T = (N + 127) // 128
+    mask = torch.zeros((Hq, T, (T + 31) // 32), dtype=torch.int32, device=dev)
+    ws = vs.workspace(max(vs.vs_block_select_workspace_size(N, w.Hkv, d),
+                          vs.vs_block_attn_workspace_size(N, Hq)), dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, N), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = {k: [] for k in ("s0", "a0", "a1")}
+
+    def step(record):
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev["s0"].append(e)
+        vs.vs_block_select(Q, K, w.alpha, mask, ws)
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev["a0"].append(e)
+        vs.vs_block_sparse_attn_fwd(Q, K, V, mask, O, lse, ws)
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev["a1"].append(e)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+    rc, flags = vs.vs_read_device_status(ws)
+    if rc != vs.VS_OK:
+        raise RuntimeError(f"device status {vs.status_string(rc)} flags {flags}")
+    mask_h = mask.cpu().numpy().view(np.uint32)
+    pairs = block_pairs(mask_h, N)
+    flops = 4.0 * d * pairs
+    dense_pairs = Hq * N * (N + 1) // 2
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            step(True)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_step = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["s0"], ev["a1"])]))
+    ms_att = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]))
+    ms_step, ms_att = max_over_ranks([ms_step, ms_att], dev)
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    dense_ms = None
+    if args.dense_steps > 0:
+        Od = torch.empty_like(Q)
+        wsd = vs.workspace(256, dev)
+        vs.vs_dense_attn_fwd(Q, K, V, Od, None, wsd)
+        ts = []
+        for _ in range(args.dense_steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            vs.vs_dense_attn_fwd(Q, K, V, Od, None, wsd)
+            b_.record(stream)
+            b_.synchronize()
+            ts.append(a.elapsed_time(b_))
+        dense_ms = float(np.mean(ts))
+        del Od
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+                      for x in (Qb, Kb, Vb))
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV))
+        d2h = hO.numel() * hO.element_size()
+        ts = []
+        for _ in range(2):
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            step(False)
+            hO.copy_(O, non_blocking=True)
+            b_.record(stream)
+            b_.synchronize()
+            ts.append(a.elapsed_time(b_))
+        e2e_ms = max_over_ranks([float(np.min(ts[1:]))], dev)[0]
+        e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+    peaks, peak_kind = measured_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    algo_bytes = (Q.numel() + K.numel() + V.numel() + O.numel()) * 2 + lse.numel() * 4
+    t_roof_ms = max(flops / (peak * 1e12), algo_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generators shaped like the pages' workloads)",
+        "config": {"workload": w.name, "N": N, "Hq": Hq, "Hkv": w.Hkv, "d": d, "alpha": w.alpha,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs exceed L2; a 256 MiB buffer is written between timed steps, "
+                         "outside the timed windows"},
+        "ms_select": round(ms_step - ms_att, 3), "ms_attention": round(ms_att, 3),
+        "selected_pairs": int(pairs), "density_vs_causal": round(pairs / dense_pairs, 5),
+        "dense_ms": None if dense_ms is None else round(dense_ms, 3),
+        "speedup_vs_dense": None if dense_ms is None else round(dense_ms / ms_step, 3),
+        "roofline": {"bound": "tensor", "achieved": round(flops / (ms_att * 1e-3) / 1e12, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(t_roof_ms / ms_att, 4),
+                     "traffic": None, "kernel": "vs_block_sparse_attn_fwd (plan + attn)",
+                     "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)"},
+        "e2e": e2e, "gpu_launches": 4 * args.steps, "input_gen_s": round(gen_s, 1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = block_oracle_sample(w, Qb, Kb, Vb, mask_h, args.cpu_seconds)
+    out["clocks"] = clk.summary()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def block_oracle_sample(w, Qb, Kb, Vb, mask, seconds, seed=0,
+                        sets_from="this run's GPU selection"):
+    """The fp64 oracle's block-sparse rows on random rows of random heads for
+    about `seconds`; effective TFLOP/s by pair count."""
+    import oracle
+    N, Hq, d = Qb.shape
+    T = mask.shape[1]
+    bits = np.unpackbits(np.ascontiguousarray(mask).view(np.uint8), bitorder="little")
+    bits = bits.reshape(mask.shape[0], T, -1)[:, :, :T].astype(bool)
+    rng = np.random.default_rng(seed)
+    t_used, p_done, rows_done = 0.0, 0, 0
+    while t_used < seconds:
+        h = int(rng.integers(0, Hq))
+        rows = np.sort(rng.integers(0, N, 32))
+        t1 = time.time()
+        oracle.attn_block_rows(Qb, Kb, Vb, h, rows, mask)
+        t_used += time.time() - t1
+        for i in rows:
+            I = i // 128
+            p_done += 128 * int(bits[h, I, :I].sum()) + (int(i - 128 * I + 1) if bits[h, I, I] else 0)
+        rows_done += rows.size
+    return {"value": round(4.0 * d * p_done / t_used / 1e12, 6), "unit": UNIT,
+            "cores": _cpu_cores(), "kind": "oracle",
+            "sample": f"{rows_done} query rows (32 random rows of a random head per draw) of "
+                      f"{w.name}, fp64 block-sparse row oracle, {t_used:.1f} s; blocks from "
+                      f"{sets_from}"}
+
+
+def run_blocks_reference(args, w):
+    """Reference arm of the block workload: the oracle's own block selection
+    (on two heads, for time) and its block-sparse rows, rank 0 only."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    Qb, Kb, Vb = w.qkv()
+    heads = [0, w.Hq // 2]
+    sel, _ = oracle.block_select(Qb, Kb, w.alpha, heads=heads)
+    T = sel.shape[1]
+    mask = np.zeros((w.Hq, T, sel.shape[2]), np.uint32)
+    mask[heads] = sel
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals, last = [], None
+    for it in range(args.warmup + args.steps):
+        # rows of the two selected heads only (their masks are the oracle's)
+        Qs = np.ascontiguousarray(Qb[:, heads])
+        Ks = np.ascontiguousarray(Kb[:, [h // (w.Hq // w.Hkv) for h in heads]])
+        last = block_oracle_sample(w, Qs, Ks, Vb[:, [h // (w.Hq // w.Hkv) for h in heads]],
+                                   mask[heads], per_step, seed=it,
+                                   sets_from="the oracle's own block selection (2 heads)")
+        if it >= args.warmup:
+            vals.append(last["value"])
+    value = float(np.mean(vals))
+    print(json.dumps({
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "impl": "reference",
+        "data": "synthetic (seeded generators shaped like the pages' workloads)",
+        "config": {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   "alpha": w.alpha},
+        "cpu_baseline": dict(last, value=round(value, 6),
+                             sample=last["sample"] + f"; {per_step:.1f} s per step"),
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def main():
     args = parse()
+    if args.workload in BLOCK_WORKLOADS:
+        wb = BLOCK_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            run_blocks_reference(args, wb)
+        else:
+            run_blocks(args, wb)
+        return
     if args.workload in BATCH_WORKLOADS:
         if args.impl == "reference":
             run_batch_reference(args, BATCH_WORKLOADS[args.workload])

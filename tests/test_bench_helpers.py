@@ -23,3 +23,25 @@ def test_dense_and_empty():
     assert bench.pairs_per_set(N, np.arange(N), []) == N * (N + 1) // 2
     assert bench.pairs_per_set(N, [], []) == 0
     assert bench.pairs_per_set(N, [], [0]) == N
+
+
+def test_block_pairs_brute_force():
+    # causal pairs inside kept blocks, against an explicit count
+    rng = np.random.default_rng(3)
+    for N in (1, 128, 300, 1000):
+        T = (N + 127) // 128
+        keep = np.tril(rng.random((2, T, T)) < 0.4)
+        keep[:, np.arange(T), np.arange(T)] = rng.random((2, T)) < 0.8
+        W = (T + 31) // 32
+        mask = np.zeros((2, T, W), np.uint32)
+        for h in range(2):
+            for I in range(T):
+                for J in range(T):
+                    if keep[h, I, J]:
+                        mask[h, I, J >> 5] |= np.uint32(1 << (J & 31))
+        want = 0
+        for h in range(2):
+            for i in range(N):
+                for j in range(i + 1):
+                    want += int(keep[h, i // 128, j // 128])
+        assert bench.block_pairs(mask, N) == want

@@ -40,6 +40,18 @@ def test_block_select_against_oracle(N, d, Hq, Hkv, alpha, cuda_device):
     assert np.array_equal(got, ref)
 
 
+@pytest.mark.slow
+def test_block_select_long_rows_recompute_path(cuda_device):
+    # T > 1024 blocks: the dot products are recomputed instead of kept
+    N = 140000
+    Qb, Kb, _ = gen_qkv(21, N, 1, 1, 64, 500000.0)
+    Qb, Kb = plant_block_structure(Qb, Kb, seed=21)
+    ref, margin = oracle.block_select(Qb, Kb, 0.3)
+    assert (margin > 1e-9).all(), margin
+    got = _gpu_mask(bf16_to_dev(Qb), bf16_to_dev(Kb), 0.3)
+    assert np.array_equal(got, ref)
+
+
 def _gpu_block_attn(Qb, Kb, Vb, mask):
     Q, K, V = (bf16_to_dev(x) for x in (Qb, Kb, Vb))
     N, Hq, d = Q.shape

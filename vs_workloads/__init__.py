@@ -351,33 +351,76 @@ BATCH_WORKLOADS = {
 
 
 def plant_block_structure(Qb: np.ndarray, Kb: np.ndarray, seed: int, sinks: int = 3,
-                          strength: float = 5.8, local: float = 4.8, period: float = 2048.0):
+                          strength: float = 5.8, local: float = 2.9, period: float = 1024.0,
+                          chunk: int = 8192):
     """Block-level attention structure on top of bf16 Q/K bits (returns new
     bits): per KV head a random unit direction u is added to every query of
     its group (x strength) and to the keys of block 0 and `sinks` random
     blocks (x strength), so those blocks act as sinks (a logit bump of about
-    strength^2 / sqrt(d)); and a slow rotation in two further directions,
-    local * (cos(w t) e1 + sin(w t) e2) with w = 2 pi / period, is added to
-    queries and keys at position t, so nearby blocks score higher (a bump of
-    about local^2 cos(w (i - j)) / sqrt(d)).  The result is rounded to bf16
-    once (round to nearest even)."""
+    strength^2 / sqrt(d)); and slow rotations in four further pairs of
+    directions, local * sum_m (cos(w_m t) e_2m + sin(w_m t) e_2m+1) with
+    periods period x (1, phi, phi^2, phi^3) (phi the golden ratio, so the
+    rotations never realign), are added to queries and keys at position t:
+    nearby blocks score higher (a bump of about
+    local^2 sum_m cos(w_m (i - j)) / sqrt(d), 4 local^2 / sqrt(d) at i = j).
+    The result is rounded to bf16 once (round to nearest even); tokens are
+    processed in chunks."""
     N, Hq, d = Qb.shape
     Hkv = Kb.shape[1]
     G = Hq // Hkv
     T = (N + 127) // 128
     rng = np.random.default_rng([seed, 7])
-    q = bf16_bits_to_f32(Qb).astype(np.float64)
-    k = bf16_bits_to_f32(Kb).astype(np.float64)
-    t = np.arange(N, dtype=np.float64)
-    w = 2.0 * np.pi / period
-    rot = np.stack([np.cos(w * t), np.sin(w * t)], 1)  # [N, 2]
+    dirs, sink_blocks = [], []
     for g in range(Hkv):
-        basis, _ = np.linalg.qr(rng.standard_normal((d, 3)))
-        u, e = basis[:, 0], basis[:, 1:3]
-        blocks = np.unique(np.concatenate([[0], rng.integers(0, T, sinks)]))
-        for J in blocks:
-            k[128 * J:128 * J + 128, g] += strength * u
-        k[:, g] += local * rot @ e.T
-        for h in range(g * G, (g + 1) * G):
-            q[:, h] += strength * u + local * rot @ e.T
-    return f64_to_bf16_bits(q), f64_to_bf16_bits(k)
+        basis, _ = np.linalg.qr(rng.standard_normal((d, 9)))
+        dirs.append((basis[:, 0], basis[:, 1:9]))
+        sink_blocks.append(np.unique(np.concatenate([[0], rng.integers(0, T, sinks)])))
+    phi = (1.0 + 5.0 ** 0.5) / 2.0
+    w = 2.0 * np.pi / (period * phi ** np.arange(4))
+    Qo = np.empty_like(Qb)
+    Ko = np.empty_like(Kb)
+    for t0 in range(0, N, chunk):
+        t1 = min(N, t0 + chunk)
+        q = bf16_bits_to_f32(Qb[t0:t1]).astype(np.float64)
+        k = bf16_bits_to_f32(Kb[t0:t1]).astype(np.float64)
+        t = np.arange(t0, t1, dtype=np.float64)
+        rot = np.stack([f(wm * t) for wm in w for f in (np.cos, np.sin)], 1)  # [n, 8]
+        blk = np.arange(t0, t1) // 128
+        for g in range(Hkv):
+            u, e = dirs[g]
+            k[np.isin(blk, sink_blocks[g]), g] += strength * u
+            k[:, g] += local * rot @ e.T
+            for h in range(g * G, (g + 1) * G):
+                q[:, h] += strength * u + local * rot @ e.T
+        Qo[t0:t1] = f64_to_bf16_bits(q)
+        Ko[t0:t1] = f64_to_bf16_bits(k)
+    return Qo, Ko
+
+
+@dataclass
+class BlockWorkload:
+    """FlashPrefill-style block-sparse prefill of one sequence: Q/K/V from the
+    seeded generator with plant_block_structure on Q and K; selection by
+    vs_block_select at `alpha`."""
+    name: str
+    N: int
+    Hq: int
+    Hkv: int
+    d: int
+    rope_base: float
+    seed: int
+    alpha: float
+    description: str = ""
+
+    def qkv(self):
+        Qb, Kb, Vb = gen_qkv(self.seed, self.N, self.Hq, self.Hkv, self.d, self.rope_base)
+        Qb, Kb = plant_block_structure(Qb, Kb, seed=self.seed)
+        return Qb, Kb, Vb
+
+
+BLOCK_WORKLOADS = {
+    "flashprefill_128k": BlockWorkload(
+        "flashprefill_128k", 131072, 32, 8, 128, 500000.0, 17, 0.3,
+        description="32q/8kv, d=128, N=131072, planted sink + local block structure, block "
+                    "pattern discovery at alpha 0.3, block-sparse attention"),
+}
