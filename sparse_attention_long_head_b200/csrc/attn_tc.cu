@@ -549,14 +549,16 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 __host__ __device__ constexpr bool poly_pair(int j) { return (j % VS_POLY_DEN) < VS_POLY_NUM; }
 
 // p = 2^(s * scale_log2 - m) for one 128-column row (s is already -inf where
-// masked), packed to bf16 pairs into pk, row sum into ls.  One call site only:
-// two inlined copies make the compiler spill the row.
+// masked), packed to bf16 pairs and stored over the row's S columns in TMEM
+// 32 columns at a time (all of S is already in registers), row sum into ls.
+// One call site only: two inlined copies make the compiler spill the row.
 __device__ __forceinline__ void exp_tile(const uint32_t (&sr)[4][32], const uint32_t (&mw)[4],
-                                         bool masked, float sl2, float m_base,
-                                         uint32_t (&pk)[2][32], float& ls) {
+                                         bool masked, float sl2, float m_base, uint32_t tS,
+                                         float& ls) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
+    uint32_t pk[16];  // P of 32 columns, stored as soon as it is formed
 #pragma unroll
     for (int c = 0; c < 32; c += 2) {
       const float x0 = fmaf(__uint_as_float(sr[q][c]), sl2, -m_base);
@@ -576,8 +578,9 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&sr)[4][32], const uint
       }
       acc[(c >> 1) & 1] += p0;
       acc[2 + ((c >> 1) & 1)] += p1;
-      pk[q >> 1][(q & 1) * 16 + c / 2] = pack_bf16x2(p0, p1);
+      pk[c / 2] = pack_bf16x2(p0, p1);
     }
+    tmem_st16(tS + 16 * q, pk);
   }
   ls = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
@@ -724,11 +727,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         const float m_base = m_use == -INFINITY ? 0.f : m_use;
         float ls = 0.f;
-        uint32_t pk[2][32];
-        exp_tile(sr, mw, masked, P.scale_log2, m_base, pk, ls);
+        exp_tile(sr, mw, masked, P.scale_log2, m_base, tS, ls);
         l += ls;
-        tmem_st32(tS, pk[0]);
-        tmem_st32(tS + 32, pk[1]);
         if (k > 0 && __any_sync(0xffffffffu, need)) {
           // O must be rescaled before PV(k) accumulates into it; PV(k-1) is
           // complete because S(k) was issued after it.

@@ -419,6 +419,9 @@ class BlockWorkload:
 
 
 BLOCK_WORKLOADS = {
+    "flashprefill_32k": BlockWorkload(
+        "flashprefill_32k", 32768, 32, 8, 128, 500000.0, 18, 0.3,
+        description="flashprefill_128k's recipe at N=32768 (the small profiling case)"),
     "flashprefill_128k": BlockWorkload(
         "flashprefill_128k", 131072, 32, 8, 128, 500000.0, 17, 0.3,
         description="32q/8kv, d=128, N=131072, planted sink + local block structure, block "
