@@ -68,7 +68,9 @@ struct ScoreArgs {
 // (x = 0..3; a warp's 32 blocks then sit 17 doubles apart in the stage, in
 // distinct banks) and probes 4 (t / 64) + {0..3} (one value per warp,
 // broadcast).  The block means stream through shared memory 16 columns at a
-// time (coalesced rows), so every loaded value feeds four fused multiply-adds.
+// time (coalesced rows; the next 16 columns are loaded into registers while
+// the current ones are used), so every loaded value feeds four fused
+// multiply-adds.
 constexpr int kJChunk = 256;
 constexpr int kCChunk = 16;
 
@@ -76,18 +78,27 @@ template <int D>
 __device__ __forceinline__ void chunk_dots(const ScoreArgs& a, const double* probes,
                                            double* kstage, int J0, int I, double (&acc)[4][4]) {
   const int tid = threadIdx.x, jg = tid % 64, pg = tid / 64;
+  // this thread stages column tid % 16 of rows J0 + tid / 16 + 16 k (k = 0..15)
+  const int cc_ld = tid % kCChunk, jj_ld = tid / kCChunk;
+  auto load = [&](int c0, double (&v)[16]) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int J = J0 + jj_ld + 16 * k;
+      v[k] = J < I ? __ldg(a.kbar + (int64_t)J * D + c0 + cc_ld) : 0.0;
+    }
+  };
 #pragma unroll
   for (int x = 0; x < 4; ++x)
 #pragma unroll
     for (int y = 0; y < 4; ++y) acc[x][y] = 0.0;
+  double nxt[16];
+  load(0, nxt);
   for (int c0 = 0; c0 < D; c0 += kCChunk) {
     __syncthreads();  // the previous stage has been read
-    for (int e = tid; e < kJChunk * kCChunk; e += kScoreThreads) {
-      const int jj = e / kCChunk, cc = e % kCChunk;
-      const int J = J0 + jj;
-      kstage[jj * (kCChunk + 1) + cc] = J < I ? __ldg(a.kbar + (int64_t)J * D + c0 + cc) : 0.0;
-    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) kstage[(jj_ld + 16 * k) * (kCChunk + 1) + cc_ld] = nxt[k];
     __syncthreads();
+    if (c0 + kCChunk < D) load(c0 + kCChunk, nxt);  // in flight while this stage is used
 #pragma unroll
     for (int cc = 0; cc < kCChunk; ++cc) {
       double pv[4], kv[4];
