@@ -115,6 +115,44 @@ def max_over_ranks(values, device=None):
     return [float(x) for x in t.tolist()]
 
 
+_CUDART = None
+
+
+def _cudart():
+    """The CUDA runtime torch already loaded (for strided asynchronous copies)."""
+    global _CUDART
+    if _CUDART is None:
+        import ctypes
+        import ctypes.util
+        path = None
+        try:
+            import nvidia.cuda_runtime as ncr
+            cand = os.path.join(list(ncr.__path__)[0], "lib", "libcudart.so.12")
+            path = cand if os.path.exists(cand) else None
+        except ImportError:
+            pass
+        lib = ctypes.CDLL(path or ctypes.util.find_library("cudart"))
+        lib.cudaMemcpy2DAsync.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                          ctypes.c_size_t, ctypes.c_size_t, ctypes.c_size_t,
+                                          ctypes.c_int, ctypes.c_void_p]
+        lib.cudaMemcpy2DAsync.restype = ctypes.c_int
+        _CUDART = lib
+    return _CUDART
+
+
+def copy_heads(dst, src, h0, h1, stream):
+    """Copy heads [h0, h1) of a token-major [N, H, d] tensor between host
+    (pinned) and device, as one strided copy on `stream`."""
+    N, H, d = src.shape
+    es = src.element_size()
+    kind = 1 if dst.is_cuda else 2  # host->device / device->host
+    rc = _cudart().cudaMemcpy2DAsync(dst.data_ptr() + h0 * d * es, H * d * es,
+                                     src.data_ptr() + h0 * d * es, H * d * es,
+                                     (h1 - h0) * d * es, N, kind, stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"cudaMemcpy2DAsync failed ({rc})")
+
+
 def sum_over_ranks(values, device=None):
     """Element-wise sum of a list of floats over all ranks (identity at world 1)."""
     import torch
@@ -411,7 +449,12 @@ def run_ours(args, w):
         agg = {"ms": float(np.mean(ts)), "row_sum_err": float((A_v.sum(1) - N).abs().max() / N)}
         del A_v, A_s, lse_d
 
-    # end to end through the public API with host buffers (pinned)
+    # End to end through the public API with host buffers (pinned): per KV
+    # group, heaviest first, its Q/K/V heads (and score rows) are copied in on
+    # one stream, its indexer / selects / attention run on the compute stream
+    # once they have landed, and its O heads are copied out on a third stream,
+    # so the copies of one group overlap the compute of another.  Heads are
+    # independent, so the result is the one-call result (checked).
     e2e = None
     if not args.no_e2e:
         hQ = torch.from_numpy(Qb.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -422,27 +465,74 @@ def run_ours(args, w):
         hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in [hQ, hK, hV] + hS)
         d2h = hO.numel() * hO.element_size()
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        G = Hq // Hkv
+        # heaviest group first (selected pairs from the warm-up's index sets):
+        # the copies of the later groups then hide under the longest compute
+        gcost = [sum(per_set[(h * H_sel) // Hq] for h in range(g * G, (g + 1) * G))
+                 for g in range(Hkv)]
+        order = sorted(range(Hkv), key=lambda g: -gcost[g])
+
+        def e2e_step():
+            start = torch.cuda.Event()
+            start.record(stream)
+            s_in.wait_event(start)
+            landed, done = {}, {}
+            for g in order:
+                h0, h1 = g * G, (g + 1) * G
+                s0, s1 = h0 * H_sel // Hq, h1 * H_sel // Hq
+                copy_heads(Q, hQ, h0, h1, s_in)
+                copy_heads(K, hK, g, g + 1, s_in)
+                copy_heads(V, hV, g, g + 1, s_in)
+                if not w.indexer:
+                    with torch.cuda.stream(s_in):
+                        LV[s0:s1].copy_(hS[0][s0:s1], non_blocking=True)
+                        LS[s0:s1].copy_(hS[1][s0:s1], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(s_in)
+                landed[g] = e
+            for g in order:
+                h0, h1 = g * G, (g + 1) * G
+                s0, s1 = h0 * H_sel // Hq, h1 * H_sel // Hq
+                stream.wait_event(landed[g])
+                if w.indexer:
+                    vs.vs_index_scores(K[:, g:g + 1], V[:, g:g + 1], W1d, W2d, LV[s0:s1], LS[s0:s1])
+                vs.vs_select(LV[s0:s1], mode, w.k_v, w.tau_v, vi[s0:s1], vc[s0:s1], ws_sel)
+                vs.vs_select(LS[s0:s1], mode, w.k_s, w.tau_s, si[s0:s1], sc[s0:s1], ws_sel2)
+                vs.vs_sparse_attn_fwd(Q[:, h0:h1], K[:, g:g + 1], V[:, g:g + 1], vi[s0:s1],
+                                      vc[s0:s1], si[s0:s1], sc[s0:s1], O[:, h0:h1], lse[h0:h1],
+                                      ws_att)
+                e = torch.cuda.Event()
+                e.record(stream)
+                done[g] = e
+            for g in order:
+                s_out.wait_event(done[g])
+                copy_heads(hO, O, g * G, (g + 1) * G, s_out)
+            stream.wait_stream(s_out)
+
         ts = []
-        for it in range(2):
+        for it in range(3):
             torch.cuda.synchronize()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            Q.copy_(hQ, non_blocking=True)
-            K.copy_(hK, non_blocking=True)
-            V.copy_(hV, non_blocking=True)
-            if not w.indexer:
-                LV.copy_(hS[0], non_blocking=True)
-                LS.copy_(hS[1], non_blocking=True)
-            step(False)
-            hO.copy_(O, non_blocking=True)
+            e2e_step()
             b.record(stream)
             b.synchronize()
             ts.append(a.elapsed_time(b))
+        # the pipelined result is the one-call result
+        O_ref = O.clone()
+        step(False)
+        torch.cuda.synchronize()
+        if not torch.equal(O, O_ref):
+            raise RuntimeError("pipelined end-to-end output differs from the one-call output")
+        del O_ref
         e2e_ms = max_over_ranks([float(np.min(ts[1:] if len(ts) > 1 else ts))], dev)[0]
         e2e = {"value": round(job_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h)}
+               "d2h_bytes_per_step": int(d2h),
+               "pipeline": "per KV group, heaviest first: copy-in stream, compute stream, "
+                           "copy-out stream"}
 
     peaks, peak_kind = measured_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
