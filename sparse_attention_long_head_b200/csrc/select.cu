@@ -425,9 +425,36 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
                           cudaStream_t stream) {
   int C = (N + 4095) / 4096;
   C = C < 1 ? 1 : (C > kSelMaxCluster ? kSelMaxCluster : C);
-  // Few heads leave most SMs idle: split long rows over 16-CTA clusters.
-  const bool wide = C == kSelMaxCluster && H * kSelMaxCluster * 2 <= device_sm_count() &&
-                    N >= 16 * 4096;
+  // Few heads leave most SMs idle: split long rows over 16-CTA clusters (a
+  // non-portable size: used only when the device can place such a cluster).
+  bool wide = C == kSelMaxCluster && H * kSelMaxCluster * 2 <= device_sm_count() &&
+              N >= 16 * 4096;
+  if (wide) {
+    const int chunk16 = (N + 15) / 16;
+    const bool cache16 = chunk16 <= kSelCacheKeys;
+    auto kern16 = cache16 ? select_kernel<true> : select_kernel<false>;
+    cudaLaunchConfig_t probe = {};
+    probe.gridDim = dim3(16, H, 1);
+    probe.blockDim = dim3(kSelThreads, 1, 1);
+    probe.dynamicSmemBytes = cache16 ? sizeof(uint32_t) * chunk16 : 0;
+    cudaLaunchAttribute pa[1];
+    pa[0].id = cudaLaunchAttributeClusterDimension;
+    pa[0].val.clusterDim.x = 16;
+    pa[0].val.clusterDim.y = 1;
+    pa[0].val.clusterDim.z = 1;
+    probe.attrs = pa;
+    probe.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaFuncSetAttribute(kern16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)probe.dynamicSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&nclusters, kern16, &probe) != cudaSuccess ||
+        nclusters < 1) {
+      cudaGetLastError();  // clear a refusal; fall back to the portable size
+      wide = false;
+    }
+  }
   if (wide) C = 16;
   const int chunk = (N + C - 1) / C;
   const bool cache = chunk <= kSelCacheKeys;
