@@ -206,3 +206,29 @@ def test_packed_and_gathered_vertical_paths_agree(cuda_device):
     for h in range(4):
         Or, lr = oracle.attn_rows(Qb, Kb, Vb, h, np.arange(N), vi, vc, si, sc)
         compare_rows(Od[:, h], Or, outs[1][1][h].cpu().numpy(), lr, what=f"packed head {h}")
+
+
+@pytest.mark.slow
+def test_maximum_sequence_length(cuda_device):
+    # N = 2^22, the largest vs_sparse_attn_fwd accepts: one head, d = 64, few
+    # keys per row; sampled rows (first / last tiles, tile boundaries, rows
+    # at and after the selected columns and offsets)
+    from vs_testutil import sample_rows
+    N, d = 1 << 22, 64
+    Qb, Kb, Vb = gen_qkv(22, N, 1, 1, d, 500000.0)
+    v = np.array([0, 5, 130, 1_000_000, 4_000_000])
+    s = np.array([0, 1, 2, 100, 127, 128, 3_000_000])
+    vi, vc = sets_to_rows([v])
+    si, sc = sets_to_rows([s])
+    Q, K, V = (bf16_to_dev(x) for x in (Qb, Kb, Vb))
+    ws = vs.workspace(vs.vs_attn_workspace_size_ld(N, 1, 1, d, vi.shape[1]))
+    O, lse = vs.sparse_attention(Q, K, V, *(torch.from_numpy(x).cuda() for x in (vi, vc, si, sc)),
+                                 ws=ws)
+    rc, flags = vs.vs_read_device_status(ws)
+    assert rc == vs.VS_OK and flags == 0
+    rows = np.unique(np.concatenate([sample_rows(N, v, seed=1, n_random=200),
+                                     v, v + 1, s, s + 1, s + 3_000_000 - s.min()]))
+    rows = rows[rows < N]
+    Or, lr = oracle.attn_rows(Qb, Kb, Vb, 0, rows, vi, vc, si, sc)
+    compare_rows(dev_to_f64(O)[rows, 0], Or, lse.cpu().numpy().astype(np.float64)[0, rows], lr,
+                 what="N = 2^22")

@@ -128,3 +128,21 @@ def test_block_prefill_pipeline(cuda_device):
     for h in range(Hq):
         Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, rows, ref)
         compare_rows(Od[rows, h], Or, lsed[h, rows], lr, what=f"pipeline head {h}")
+
+
+@pytest.mark.slow
+def test_maximum_length_block_path(cuda_device):
+    # N = 2^18, the largest the block calls accept (2048 blocks: the
+    # recompute path of the scores)
+    from vs_testutil import sample_rows
+    N = 1 << 18
+    Qb, Kb, Vb = gen_qkv(23, N, 1, 1, 64, 500000.0)
+    Qb, Kb = plant_block_structure(Qb, Kb, seed=23)
+    ref, margin = oracle.block_select(Qb, Kb, 0.3)
+    assert (margin > 1e-9).all(), margin
+    assert np.array_equal(_gpu_mask(bf16_to_dev(Qb), bf16_to_dev(Kb), 0.3), ref)
+    O, lse = _gpu_block_attn(Qb, Kb, Vb, ref)
+    rows = sample_rows(N, seed=2, n_random=200)
+    Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, 0, rows, ref)
+    compare_rows(dev_to_f64(O)[rows, 0], Or, lse.cpu().numpy().astype(np.float64)[0, rows], lr,
+                 what="block N = 2^18")

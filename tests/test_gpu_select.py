@@ -120,3 +120,14 @@ def test_maxfrac_near_uniform_long_rows(cuda_device):
     big = rng.standard_normal((2, 300000)).astype(np.float32)  # beyond the shared cache
     check_select(big, MAXF, 300000, 0.05)
     check_select(big, MAXF, 1000, 0.05)
+
+
+@pytest.mark.slow
+def test_maximum_row_length(cuda_device):
+    # N = 2^20, the largest vs_select accepts
+    rng = np.random.default_rng(20)
+    N = 1 << 20
+    s = rng.standard_normal((2, N)).astype(np.float32)
+    check_select(s, TOPK, 1000)
+    check_select(s, THR, N, 0.5)
+    check_select(s, MAXF, 5000, 0.02)
