@@ -223,7 +223,10 @@ vs_status vs_dense_attn_fwd_varlen(const void* Q, const void* K, const void* V, 
  *   mask     uint32 [Hq][T][W] output (device), T = ceil(N / 128),
  *            W = ceil(T / 32): bit J of row (h, I) set iff block J is kept.
  *   ws       at least vs_block_select_workspace_size(N, Hkv, d) bytes,
- *            256-byte aligned (status word, then the fp64 block means).
+ *            256-byte aligned: status word and work counter, the fp64 block
+ *            means, and one dot-product scratch per SM of the current device
+ *            (the size depends on that device; a workspace sized on a device
+ *            with fewer SMs fails the check with VS_ERR_WORKSPACE).
  */
 size_t vs_block_select_workspace_size(int N, int Hkv, int d);
 vs_status vs_block_select(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,

@@ -332,7 +332,8 @@ vs_status vs_block_select(const void* Q, const void* K, vs_dtype dtype, int N, i
   a.mask = mask;
   a.ws = ws;
   a.stream = stream;
-  if (cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  // status word and the kernel's work-item counter
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return VS_ERR_CUDA;
   return launch_block_select(a) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
 }
 

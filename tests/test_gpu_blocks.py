@@ -146,3 +146,24 @@ def test_maximum_length_block_path(cuda_device):
     Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, 0, rows, ref)
     compare_rows(dev_to_f64(O)[rows, 0], Or, lse.cpu().numpy().astype(np.float64)[0, rows], lr,
                  what="block N = 2^18")
+
+
+@pytest.mark.slow
+def test_flashprefill_32k_workload_full_size(cuda_device):
+    # the bench's configuration: 32 query heads over 8 KV heads (four query
+    # heads share a CTA), N = 32768; bit-exact masks for every head, and the
+    # block-sparse rows of two heads sampled
+    from vs_testutil import sample_rows
+    from vs_workloads import BLOCK_WORKLOADS
+    w = BLOCK_WORKLOADS["flashprefill_32k"]
+    Qb, Kb, Vb = w.qkv()
+    ref, margin = oracle.block_select(Qb, Kb, w.alpha)
+    assert (margin > 1e-9).all(), margin
+    got = _gpu_mask(bf16_to_dev(Qb), bf16_to_dev(Kb), w.alpha)
+    assert np.array_equal(got, ref)
+    O, lse = _gpu_block_attn(Qb, Kb, Vb, ref)
+    rows = sample_rows(w.N, seed=3, n_random=150)
+    for h in (0, 29):
+        Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, rows, ref)
+        compare_rows(dev_to_f64(O)[rows, h], Or, lse[h].cpu().numpy().astype(np.float64)[rows], lr,
+                     what=f"flashprefill_32k head {h}")
