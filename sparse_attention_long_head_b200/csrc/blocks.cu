@@ -45,12 +45,12 @@ constexpr int kProbes = 16;
 constexpr int kProbeStride = 8;
 constexpr int kMaxBlocks = 2048;     // T <= 2048 (N <= 2^18)
 constexpr int kBsWarps = 8;          // consumer (MMA) warps
-constexpr int kBsThreads = 32 * (kBsWarps + 1);
-constexpr int kBsStages = 4;         // shared-memory ring (a multiple of every stage-class count)
+constexpr int kBsThreads = 32 * (kBsWarps + 1);  // + the producer warp
 constexpr int kTilesPerStage = 2;    // 16-block tiles per stage
 constexpr int kPadBlocks = 16 * kTilesPerStage;
 constexpr size_t kCounterOffset = 128;  // work-item counter, inside the status block
 constexpr size_t kOneCtaSmem = 120 * 1024;
+constexpr size_t kMaxDynSmem = 216 * 1024;  // with the static part, under the 227 KB opt-in limit
 
 __host__ __device__ constexpr int pad_blocks(int T) { return (T + kPadBlocks - 1) / kPadBlocks * kPadBlocks; }
 
@@ -112,6 +112,7 @@ struct ScoreArgs {
   const void* Q;
   int dtype, N, Hq, Hkv, T, W, Tp, HC;  // HC: query heads per work item (1, 2 or 4)
   int n_items, n_chunks;                // items: (query block, chunk of HC heads)
+  int stages;                           // ring slots: 3, or 4 with two stage classes
   int64_t q_stride;
   double scale, alpha;
   const double* kbar;  // operand layout, [Hkv][Tp / 16 tiles]
@@ -123,29 +124,23 @@ struct ScoreArgs {
   uint64_t wait_limit_ns;
 };
 
-// Online (max, sum of exp(x - max)) merge; symmetric in its two operands, so
-// both lanes of a butterfly step end with identical values.
-__device__ __forceinline__ void lse_merge(double& m1, double& z1, double m2, double z2) {
-  const double mn = fmax(m1, m2);
-  if (mn == -INFINITY) return;
-  z1 = (m1 == -INFINITY ? 0.0 : z1 * exp(m1 - mn)) + (m2 == -INFINITY ? 0.0 : z2 * exp(m2 - mn));
-  m1 = mn;
-}
-
-// Persistent: one CTA per SM takes work items (query block I, chunk of HC
-// query heads), heaviest rows first, from a global counter.  Per item:
-//   pass 1 (MMA): each consumer warp owns one n-tile (8 probes), one or
-//     both tiles of each stage, and a class of stages (every stage when four
-//     heads share an item, else every other stage with one tile per warp at
-//     one head per item); the MMAs of its next stage are issued
-//     before the epilogue of the current one, which updates the probes'
-//     online (max, sum of exponentials) and stores the scaled dot products
-//     in the CTA's scratch (L2-resident, read back by the same lanes);
-//   pass 2 (no MMA): the normalised exponentials from the scratch, summed
-//     over each head's 16 probes, give the block scores in shared memory;
-//   then each head's maximum, threshold and mask row.
-// TPW: 16-block tiles of a stage per warp -- 2 when an item has 8 n-tiles
-// (four heads), else 1 (the stage's two tiles go to two warps).
+// Persistent: one CTA per SM; work items are (query block I, chunk of HC
+// query heads), heaviest rows first, claimed from a global counter by the
+// producer warp, which also stages each item's probe rows (raw input type)
+// and streams its block means through the ring, so the next item's data
+// arrives while the consumers finish the current one.  Per item the eight
+// consumer warps run:
+//   pass 1 (MMA): each warp owns one n-tile (8 probes), one or both tiles
+//     of each stage and a class of stages (every stage when four heads share
+//     an item; else the stage's two tiles go to two warps, and at one head
+//     per item every other stage); the MMAs of its next stage are issued
+//     before the epilogue of the current one, which stores the scaled dot
+//     products in the CTA's scratch and keeps the probes' running maxima;
+//   pass 2: e = exp(s - max) back into the scratch, and the sums Z;
+//   pass 3: the scores sum_p e / Z_p over each head's 16 probes (two
+//     addends, one per n-tile, per block), then each head's maximum,
+//     threshold and mask row.  Every scratch entry is written and read back
+//     by the same lane, so the passes need no fence.
 template <int D, int TPW>
 __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreArgs a) {
   constexpr int KS = D / 16;
@@ -153,62 +148,113 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
   constexpr int kStageDoubles = kTilesPerStage * kTileDoubles;
   constexpr uint32_t kStageBytes = sizeof(double) * kStageDoubles;
   constexpr int kCons = kBsWarps * 32;
+  constexpr int TS = kTilesPerStage / TPW;  // warps sharing a stage's tiles
+  constexpr int PF = 2;                     // scratch prefetch depth, in stages
   extern __shared__ __align__(128) double dyn[];
-  double* ring = dyn;                                 // kBsStages stages
-  double* score = ring + kBsStages * kStageDoubles;   // [HC][T]
-  __shared__ __align__(8) uint64_t full_bar[kBsStages], empty_bar[kBsStages];
-  __shared__ double part_m[kBsWarps][4 * kProbes], part_z[kBsWarps][4 * kProbes];
+  const int NT = 2 * a.HC, WPN = kBsWarps / NT, SR = WPN / TS;
+  // ring | bfrag | score: the two double2-accessed buffers first, so that
+  // both start on 16-byte boundaries whatever HC * T is
+  double* ring = dyn;  // a.stages slots
+  // the item's probes as B fragments: per (n-tile, k-step) 2 x [32 lanes][2]
+  // doubles, entry (j, lane = 4 g + t, e) = probe 8 (nt % 2) + g of head nt / 2
+  // at dimension 16 ks + t + 4 (2 j + e)
+  double* bfrag = ring + a.stages * kStageDoubles;
+  double* score = bfrag + NT * KS * 128;  // [HC][T]
+  __shared__ __align__(8) uint64_t full_bar[4], empty_bar[4], pfull_bar, pempty_bar;
+  __shared__ double part[kBsWarps][4 * kProbes];
   __shared__ double st_m[4 * kProbes], st_rz[4 * kProbes];
-  __shared__ double red[kBsWarps];
-  __shared__ int item_buf[2];
+  __shared__ double red[kBsWarps][4];
+  __shared__ int item_slot;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // n-tiles; warps per n-tile; warps splitting a stage's tiles; stage
-  // classes (stage q is consumed by the warps of class q % SR, and since SR
-  // divides kBsStages each ring slot serves one class, whose warps wait for
-  // the slot's phases in order)
-  constexpr int TS = kTilesPerStage / TPW;
-  const int NT = 2 * a.HC, WPN = kBsWarps / NT, SR = WPN / TS;
   if (tid == 0) {
-    for (int s = 0; s < kBsStages; ++s) {
+    for (int s = 0; s < a.stages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), NT * TS);
     }
+    mbar_init(smem_u32(&pfull_bar), 1);
+    mbar_init(smem_u32(&pempty_bar), kBsWarps);
     abort_flag = 0;
     fence_mbar_init();
   }
+  __syncthreads();
   const WaitCtx wc{a.wait_limit_ns, a.status, &abort_flag};
-  double* scr = a.scratch + (int64_t)blockIdx.x * a.scratch_doubles;
-  int s0 = 0;      // stages issued / consumed before the current item
-  int issued = 0;  // producer: stages whose copies were issued
-  bool ok = true;  // this thread's bounded waits all succeeded
-  for (int it = 0;; ++it) {
-    if (tid == 0) item_buf[it & 1] = atomicAdd(a.counter, 1);
-    if (__syncthreads_or(!ok)) break;
-    const int k = item_buf[it & 1];
-    if (k >= a.n_items) break;
-    const int I = a.T - 1 - k / a.n_chunks;
-    const int h0 = (k % a.n_chunks) * a.HC;
-    const int g = h0 / (a.Hq / a.Hkv);
-    if (I == 0) {  // no earlier block: the diagonal alone
-      for (int e = tid; e < a.HC * a.W; e += blockDim.x) {
-        const int hl = e / a.W, w = e % a.W;
-        a.mask[((int64_t)(h0 + hl) * a.T) * a.W + w] = w == 0 ? 1u : 0u;
-      }
-      continue;
-    }
-    int np = 0;
+  const int esz = a.dtype == VS_BF16 ? 2 : 4;
+  auto item_rows = [&](int k, int& I, int& h0, int& np, int& nsq) {
+    I = a.T - 1 - k / a.n_chunks;
+    h0 = (k % a.n_chunks) * a.HC;
+    np = 0;
     while (np < kProbes && 128 * (int64_t)I + kProbeStride * np < a.N) ++np;
-    const int nsq = (I + 16 * kTilesPerStage - 1) / (16 * kTilesPerStage);  // stages
-    const int sb = s0;
-    s0 += nsq;
+    nsq = (I + 16 * kTilesPerStage - 1) / (16 * kTilesPerStage);  // 0 for I = 0
+  };
 
-    if (warp == kBsWarps) {  // producer
+  // ------------------------------------------------------------- producer
+  if (warp == kBsWarps) {
+    int s = 0;  // stages issued
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      int k = 0;
+      if (lane == 0) k = atomicAdd(a.counter, 1);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      // the fragment buffer is free once every consumer warp is past the last item's MMAs
+      if (it > 0) {
+        bool w = lane == 0 ? mbar_wait(smem_u32(&pempty_bar), (it - 1) & 1, wc) : true;
+        if (!__shfl_sync(0xffffffffu, (int)w, 0)) break;
+      }
+      int I = 0, h0 = 0, np = 0, nsq = 0;
+      if (k < a.n_items) {
+        item_rows(k, I, h0, np, nsq);
+        if (I > 0) {
+          // Probe rows (the HC heads' D values are contiguous and 16-byte
+          // aligned) in 16-byte pieces, eight per lane in flight, scattered
+          // into fragment order; rows past the probes are zeros.
+          const int per = 16 / esz;                  // elements per piece
+          const int pieces = a.HC * D / per;         // per probe row
+          for (int e0 = 0; e0 < kProbes * pieces; e0 += 8 * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const int e = e0 + 32 * x + lane, p = e / pieces;
+              v[x] = make_uint4(0u, 0u, 0u, 0u);
+              if (e < kProbes * pieces && p < np)
+                v[x] = __ldg(reinterpret_cast<const uint4*>(
+                                 static_cast<const uint8_t*>(a.Q) +
+                                 ((128 * (int64_t)I + kProbeStride * p) * a.q_stride +
+                                  (int64_t)h0 * D) * esz) + e % pieces);
+            }
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const int e = e0 + 32 * x + lane;
+              if (e >= kProbes * pieces) continue;
+              const int p = e / pieces, c0 = (e % pieces) * per;
+              const uint32_t w[4] = {v[x].x, v[x].y, v[x].z, v[x].w};
+              auto put = [&](int c, double val) {
+                const int hl = c / D, dim = c % D;
+                const int nt = 2 * hl + (p >> 3), cc = dim & 15, i = cc >> 2;
+                bfrag[(nt * KS + (dim >> 4)) * 128 + (i >> 1) * 64 + (4 * (p & 7) + (cc & 3)) * 2 +
+                      (i & 1)] = val;
+              };
+              if (esz == 2) {
+#pragma unroll
+                for (int y = 0; y < 8; ++y)  // bf16 -> fp32 is exact
+                  put(c0 + y, (double)__uint_as_float(((w[y >> 1] >> (16 * (y & 1))) & 0xffffu) << 16));
+              } else {
+#pragma unroll
+                for (int y = 0; y < 4; ++y) put(c0 + y, (double)__uint_as_float(w[y]));
+              }
+            }
+          }
+        }
+      }
+      if (lane == 0) item_slot = k;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&pfull_bar));  // release: the fragments and the item
+      if (k >= a.n_items) break;
       if (lane == 0) {
-        const double* src = a.kbar + (int64_t)g * (a.Tp / 16) * kTileDoubles;
-        for (int q = 0; q < nsq && ok; ++q) {
-          const int s = sb + q, slot = s % kBsStages, use = s / kBsStages;
+        const double* src = a.kbar + (int64_t)(h0 / (a.Hq / a.Hkv)) * (a.Tp / 16) * kTileDoubles;
+        for (int q = 0; q < nsq; ++q, ++s) {
+          const int slot = s % a.stages, use = s / a.stages;
           if (use > 0 && !mbar_wait(smem_u32(&empty_bar[slot]), (use - 1) & 1, wc)) {
             ok = false;
             break;
@@ -216,33 +262,53 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
           mbar_arrive_expect_tx(smem_u32(&full_bar[slot]), kStageBytes);
           bulk_load(smem_u32(ring + slot * kStageDoubles), src + (int64_t)q * kStageDoubles,
                     kStageBytes, smem_u32(&full_bar[slot]));
-          issued = s + 1;
         }
+      }
+      ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+    }
+    // copies still in flight (after an abort) land before the CTA exits
+    if (lane == 0)
+      for (int x = max(0, s - a.stages); x < s; ++x)
+        mbar_wait_drain(smem_u32(&full_bar[x % a.stages]), (x / a.stages) & 1, a.wait_limit_ns);
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int nt = warp % NT, sub = warp / NT;
+  const int m0 = (sub % TS) * TPW, cls = sub / TS;  // first tile of a stage; stage class
+  const int hl = nt >> 1, pb = 8 * (nt & 1);
+  const int gq = lane >> 2, t = lane & 3;
+  double* scr = a.scratch + (int64_t)blockIdx.x * a.scratch_doubles;
+  // scratch: per (stage, n-tile, tile) 2 x [32 lanes] double2 (a lane's 4 values)
+  auto scr_at = [&](int q, int m) {
+    return reinterpret_cast<double2*>(scr + (((int64_t)q * NT + nt) * kTilesPerStage + m) * 128) +
+           lane;
+  };
+  int s0 = 0;  // stages consumed before the current item
+  for (int it = 0;; ++it) {
+    bool ok = mbar_wait(smem_u32(&pfull_bar), it & 1, wc);
+    if (!named_bar_and(1, kCons, ok)) break;
+    const int k = item_slot;
+    if (k >= a.n_items) break;
+    int I, h0, np, nsq;
+    item_rows(k, I, h0, np, nsq);
+    const int sb = s0;
+    s0 += nsq;
+    if (I == 0) {  // no earlier block: the diagonal alone
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&pempty_bar));
+      for (int e = tid; e < a.HC * a.W; e += kCons) {
+        const int x = e / a.W, w = e % a.W;
+        a.mask[((int64_t)(h0 + x) * a.T) * a.W + w] = w == 0 ? 1u : 0u;
       }
       continue;
     }
-
-    // ---------------------------------------------------------- consumers
-    const int nt = warp % NT, sub = warp / NT;
-    const int m0 = (sub % TS) * TPW, cls = sub / TS;  // first tile of the stage; stage class
-    const int hl = nt >> 1, pb = 8 * (nt & 1);
-    const int gq = lane >> 2, t = lane & 3;
-    double bq[KS][4];  // B fragments: probe pb + gq of head h0 + hl
-    {
-      const int p = pb + gq;
-      const int64_t base =
-          (128 * (int64_t)I + kProbeStride * p) * a.q_stride + (int64_t)(h0 + hl) * D;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          bq[ks][i] = p < np ? load_kv(a.Q, a.dtype, base + 16 * ks + t + 4 * i) : 0.0;
-    }
+    const double2* bsrc = reinterpret_cast<const double2*>(bfrag + nt * KS * 128) + lane;
     // Issues stage q's MMAs into acc[u] (block 16 (2 q + m0 + u) + gq + 8 (i / 2),
     // probe pb + 2 t + i % 2) and releases the stage's slot.
     auto issue = [&](int q, double (&acc)[TPW][4]) -> bool {
-      const int s = sb + q, slot = s % kBsStages;
-      if (!mbar_wait(smem_u32(&full_bar[slot]), (s / kBsStages) & 1, wc)) return false;
+      const int s = sb + q, slot = s % a.stages;
+      if (!mbar_wait(smem_u32(&full_bar[slot]), (s / a.stages) & 1, wc)) return false;
       const double* sA = ring + slot * kStageDoubles;
 #pragma unroll
       for (int u = 0; u < TPW; ++u)
@@ -250,6 +316,8 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
         for (int i = 0; i < 4; ++i) acc[u][i] = 0.0;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
+        const double2 b01 = bsrc[ks * 64], b23 = bsrc[ks * 64 + 32];
+        const double bf[4] = {b01.x, b01.y, b23.x, b23.y};
 #pragma unroll
         for (int u = 0; u < TPW; ++u) {
           const double2* src =
@@ -261,23 +329,17 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
             af[2 * j] = x.x;
             af[2 * j + 1] = x.y;
           }
-          dmma_16816(acc[u], af, bq[ks]);
+          dmma_16816(acc[u], af, bf);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty_bar[slot]));  // release orders the reads
       return true;
     };
-    // scratch: per (stage, n-tile, tile) 2 x [32 lanes] double2 (a lane's 4
-    // values); each entry is written and read back by the same lane
-    auto scr_at = [&](int q, int m) {
-      return reinterpret_cast<double2*>(scr + (((int64_t)q * NT + nt) * kTilesPerStage + m) * 128) +
-             lane;
-    };
+    const bool pv0 = pb + 2 * t < np, pv1 = pb + 2 * t + 1 < np;  // this thread's probe columns
 
-    // Pass 1: online maximum and sum of exponentials of this thread's two
-    // probe columns; the dot products go to the scratch.
-    double mr[2] = {-INFINITY, -INFINITY}, zr[2] = {0.0, 0.0};
+    // Pass 1: the dot products into the scratch, and the running maxima.
+    double mr[2] = {-INFINITY, -INFINITY};
     {
       double cur[TPW][4], nxt[TPW][4];
       int q = cls;
@@ -298,17 +360,13 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
           dst[0] = make_double2(v[0], v[1]);
           dst[32] = make_double2(v[2], v[3]);
           const int J0 = 16 * (kTilesPerStage * q + m) + gq, J1 = J0 + 8;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            if (pb + 2 * t + c >= np) continue;
-            const bool oa = J0 < I, ob = J1 < I;
-            const double tm = fmax(oa ? v[c] : -INFINITY, ob ? v[2 + c] : -INFINITY);
-            if (tm > mr[c]) {
-              zr[c] = mr[c] == -INFINITY ? 0.0 : zr[c] * exp(mr[c] - tm);
-              mr[c] = tm;
-            }
-            if (oa) zr[c] += exp(v[c] - mr[c]);
-            if (ob) zr[c] += exp(v[2 + c] - mr[c]);
+          if (J0 < I) {
+            if (pv0) mr[0] = fmax(mr[0], v[0]);
+            if (pv1) mr[1] = fmax(mr[1], v[1]);
+          }
+          if (J1 < I) {
+            if (pv0) mr[0] = fmax(mr[0], v[2]);
+            if (pv1) mr[1] = fmax(mr[1], v[3]);
           }
         }
 #pragma unroll
@@ -317,111 +375,145 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
           for (int i = 0; i < 4; ++i) cur[u][i] = nxt[u][i];
       }
     }
-    // over the 8 lanes that share a column, then over the warps of the n-tile
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&pempty_bar));  // this warp's MMAs are issued
+    // maxima over the 8 lanes sharing a column, then over the n-tile's warps
 #pragma unroll
     for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1)
-        lse_merge(mr[c], zr[c], __shfl_xor_sync(0xffffffffu, mr[c], o),
-                  __shfl_xor_sync(0xffffffffu, zr[c], o));
-    if (gq == 0) {  // one partial per warp of the n-tile
+      for (int o = 4; o < 32; o <<= 1) mr[c] = fmax(mr[c], __shfl_xor_sync(0xffffffffu, mr[c], o));
+    if (gq == 0) {
+      part[sub][hl * kProbes + pb + 2 * t] = mr[0];
+      part[sub][hl * kProbes + pb + 2 * t + 1] = mr[1];
+    }
+    if (!named_bar_and(1, kCons, ok)) break;
+    if (tid < a.HC * kProbes) {
+      double m = part[0][tid];
+      for (int w = 1; w < WPN; ++w) m = fmax(m, part[w][tid]);
+      st_m[tid] = m;
+    }
+    named_bar_sync(1, kCons);
+
+    // Streams this warp's scratch entries (stages q = cls, cls + SR, ...)
+    // with PF stages in flight, calling f(q, m, v[4]) per tile and storing v
+    // back when `wb`.
+    auto sweep = [&](bool wb, auto&& f) {
+      double2 buf[PF][2 * TPW];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        part_m[sub][hl * kProbes + pb + 2 * t + c] = mr[c];
-        part_z[sub][hl * kProbes + pb + 2 * t + c] = zr[c];
+      for (int x = 0; x < PF; ++x) {
+        const int q = cls + x * SR;
+        if (q < nsq)
+#pragma unroll
+          for (int u = 0; u < TPW; ++u) {
+            buf[x][2 * u] = scr_at(q, m0 + u)[0];
+            buf[x][2 * u + 1] = scr_at(q, m0 + u)[32];
+          }
+      }
+      for (int q = cls; q < nsq; q += SR) {
+#pragma unroll
+        for (int u = 0; u < TPW; ++u) {
+          double v[4] = {buf[0][2 * u].x, buf[0][2 * u].y, buf[0][2 * u + 1].x,
+                         buf[0][2 * u + 1].y};
+          f(q, m0 + u, v);
+          if (wb) {
+            scr_at(q, m0 + u)[0] = make_double2(v[0], v[1]);
+            scr_at(q, m0 + u)[32] = make_double2(v[2], v[3]);
+          }
+        }
+#pragma unroll
+        for (int x = 0; x + 1 < PF; ++x)
+#pragma unroll
+          for (int j = 0; j < 2 * TPW; ++j) buf[x][j] = buf[x + 1][j];
+        const int qn = q + PF * SR;
+        if (qn < nsq)
+#pragma unroll
+          for (int u = 0; u < TPW; ++u) {
+            buf[PF - 1][2 * u] = scr_at(qn, m0 + u)[0];
+            buf[PF - 1][2 * u + 1] = scr_at(qn, m0 + u)[32];
+          }
+      }
+    };
+
+    // Pass 2: e = exp(s - max) (0 outside J < I or past the probes) and Z.
+    {
+      const double pm0 = st_m[hl * kProbes + pb + 2 * t], pm1 = st_m[hl * kProbes + pb + 2 * t + 1];
+      double z0 = 0.0, z1 = 0.0;
+      sweep(true, [&](int q, int m, double (&v)[4]) {
+        const int J0 = 16 * (kTilesPerStage * q + m) + gq, J1 = J0 + 8;
+        v[0] = pv0 && J0 < I ? exp(v[0] - pm0) : 0.0;
+        v[1] = pv1 && J0 < I ? exp(v[1] - pm1) : 0.0;
+        v[2] = pv0 && J1 < I ? exp(v[2] - pm0) : 0.0;
+        v[3] = pv1 && J1 < I ? exp(v[3] - pm1) : 0.0;
+        z0 += v[0] + v[2];
+        z1 += v[1] + v[3];
+      });
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        z0 += __shfl_xor_sync(0xffffffffu, z0, o);
+        z1 += __shfl_xor_sync(0xffffffffu, z1, o);
+      }
+      if (gq == 0) {
+        part[sub][hl * kProbes + pb + 2 * t] = z0;
+        part[sub][hl * kProbes + pb + 2 * t + 1] = z1;
       }
     }
     for (int e = tid; e < a.HC * I; e += kCons) score[(e / I) * a.T + e % I] = 0.0;
-    ok = named_bar_and(1, kCons, ok);
-    if (!ok) continue;
+    named_bar_sync(1, kCons);
     if (tid < a.HC * kProbes) {
-      double m = part_m[0][tid], z = part_z[0][tid];
-      for (int w = 1; w < WPN; ++w) lse_merge(m, z, part_m[w][tid], part_z[w][tid]);
-      st_m[tid] = m;
+      double z = part[0][tid];
+      for (int w = 1; w < WPN; ++w) z += part[w][tid];
       st_rz[tid] = 1.0 / z;
     }
     named_bar_sync(1, kCons);
 
-    // Pass 2: Score(I, J) sums, two addends (one per n-tile) per (head, J).
+    // Pass 3: block scores (sums over the probes; the mean's 1/np cancels
+    // in the comparison with alpha times the best).
     {
-      double pm[2], prz[2];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        pm[c] = st_m[hl * kProbes + pb + 2 * t + c];
-        prz[c] = st_rz[hl * kProbes + pb + 2 * t + c];
-      }
-      double2 cur[2 * TPW], nxt[2 * TPW];
-      int q = cls;
-      if (q < nsq) {
-#pragma unroll
-        for (int u = 0; u < TPW; ++u) {
-          cur[2 * u] = scr_at(q, m0 + u)[0];
-          cur[2 * u + 1] = scr_at(q, m0 + u)[32];
-        }
-      }
-      for (; q < nsq; q += SR) {
-        const int qn = q + SR;
-        if (qn < nsq) {
-#pragma unroll
-          for (int u = 0; u < TPW; ++u) {
-            nxt[2 * u] = scr_at(qn, m0 + u)[0];
-            nxt[2 * u + 1] = scr_at(qn, m0 + u)[32];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < TPW; ++u) {
-          const int m = m0 + u;
-          const double v[4] = {cur[2 * u].x, cur[2 * u].y, cur[2 * u + 1].x, cur[2 * u + 1].y};
-          const int J0 = 16 * (kTilesPerStage * q + m) + gq, J1 = J0 + 8;
-          double ra = 0.0, rb = 0.0;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            if (pb + 2 * t + c >= np) continue;
-            if (J0 < I) ra += exp(v[c] - pm[c]) * prz[c];
-            if (J1 < I) rb += exp(v[2 + c] - pm[c]) * prz[c];
-          }
-          ra += __shfl_xor_sync(0xffffffffu, ra, 1);
-          ra += __shfl_xor_sync(0xffffffffu, ra, 2);
-          rb += __shfl_xor_sync(0xffffffffu, rb, 1);
-          rb += __shfl_xor_sync(0xffffffffu, rb, 2);
-          // 0 + x is exact and x + y == y + x, so the order of the two
-          // n-tiles' additions does not change the sum
-          if (t == 0 && J0 < I) atomicAdd(&score[hl * a.T + J0], ra);
-          if (t == 0 && J1 < I) atomicAdd(&score[hl * a.T + J1], rb);
-        }
-#pragma unroll
-        for (int j = 0; j < 2 * TPW; ++j) cur[j] = nxt[j];
-      }
+      const double r0 = pv0 ? st_rz[hl * kProbes + pb + 2 * t] : 0.0;
+      const double r1 = pv1 ? st_rz[hl * kProbes + pb + 2 * t + 1] : 0.0;
+      sweep(false, [&](int q, int m, double (&v)[4]) {
+        const int J0 = 16 * (kTilesPerStage * q + m) + gq, J1 = J0 + 8;
+        double ra = v[0] * r0 + v[1] * r1, rb = v[2] * r0 + v[3] * r1;
+        ra += __shfl_xor_sync(0xffffffffu, ra, 1);
+        ra += __shfl_xor_sync(0xffffffffu, ra, 2);
+        rb += __shfl_xor_sync(0xffffffffu, rb, 1);
+        rb += __shfl_xor_sync(0xffffffffu, rb, 2);
+        // 0 + x is exact and x + y == y + x, so the order of the two
+        // n-tiles' additions does not change the sum
+        if (t == 0 && J0 < I) atomicAdd(&score[hl * a.T + J0], ra);
+        if (t == 0 && J1 < I) atomicAdd(&score[hl * a.T + J1], rb);
+      });
     }
     named_bar_sync(1, kCons);
 
-    // Threshold and bitmask, head by head.
+    // Threshold and bitmask rows of the item's heads.
+    double best[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int J = tid; J < I; J += kCons)
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        if (x < a.HC) best[x] = fmax(best[x], score[x * a.T + J]);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) best[x] = fmax(best[x], __shfl_xor_sync(0xffffffffu, best[x], o));
+      if (lane == 0) red[warp][x] = best[x];
+    }
+    named_bar_sync(1, kCons);
     for (int x = 0; x < a.HC; ++x) {
+      double b = red[0][x];
+#pragma unroll
+      for (int w = 1; w < kBsWarps; ++w) b = fmax(b, red[w][x]);
+      const double thr = a.alpha * b;
       const double* sc = score + x * a.T;
-      double best = 0.0;
-      for (int J = tid; J < I; J += kCons) best = fmax(best, sc[J] / (double)np);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
-      if (lane == 0) red[warp] = best;
-      named_bar_sync(1, kCons);
-      best = red[0];
-#pragma unroll
-      for (int w = 1; w < kBsWarps; ++w) best = fmax(best, red[w]);
-      const double thr = a.alpha * best;
       uint32_t* out = a.mask + ((int64_t)(h0 + x) * a.T + I) * a.W;
       for (int w = warp; w < a.W; w += kBsWarps) {
         const int J = 32 * w + lane;
-        const bool keep = J == I || (J < I && sc[J] / (double)np >= thr);
+        const bool keep = J == I || (J < I && sc[J] >= thr);
         const uint32_t bits = __ballot_sync(0xffffffffu, keep);
         if (lane == 0) out[w] = bits;
       }
-      named_bar_sync(1, kCons);  // red[] and score[] are reused
     }
   }
-  // copies still in flight (after an abort) land before the CTA exits
-  if (warp == kBsWarps && lane == 0)
-    for (int x = max(0, issued - kBsStages); x < issued; ++x)
-      mbar_wait_drain(smem_u32(&full_bar[x % kBsStages]), (x / kBsStages) & 1, a.wait_limit_ns);
 }
 
 int num_sms() {
@@ -477,10 +569,18 @@ cudaError_t launch_block_select(const BlockSelectArgs& a) {
   s.status = static_cast<int*>(a.ws);
   s.counter = reinterpret_cast<int*>(base + kCounterOffset);
   s.wait_limit_ns = kDefaultWaitLimitNs;
+  const int NT = 2 * HC, TS = HC == 4 ? 1 : 2, SR = kBsWarps / NT / TS;
+  // ring slots: a multiple of the stage-class count SR, as many as fit
+  auto dyn_bytes = [&](int stages) {
+    return sizeof(double) * ((size_t)stages * kTilesPerStage * 16 * a.d + (size_t)HC * T +
+                             (size_t)NT * a.d * 8);
+  };
+  s.stages = SR == 1 ? 3 : 4;
+  if (dyn_bytes(s.stages) > kMaxDynSmem) s.stages = 2;
+  const size_t need = dyn_bytes(s.stages);
+  if (need > kMaxDynSmem) return cudaErrorInvalidValue;
   // more than half of an SM's shared memory: one CTA per SM, so a CTA's
   // scratch slot (its block index) is never shared
-  const size_t need =
-      sizeof(double) * ((size_t)kBsStages * kTilesPerStage * 16 * a.d + (size_t)HC * T);
   const size_t smem = need > kOneCtaSmem ? need : kOneCtaSmem;
   auto kern = a.d == 128 ? (HC == 4 ? block_score_kernel<128, 2> : block_score_kernel<128, 1>)
                          : (HC == 4 ? block_score_kernel<64, 2> : block_score_kernel<64, 1>);

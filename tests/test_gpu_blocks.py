@@ -167,3 +167,19 @@ def test_flashprefill_32k_workload_full_size(cuda_device):
         Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, rows, ref)
         compare_rows(dev_to_f64(O)[rows, h], Or, lse[h].cpu().numpy().astype(np.float64)[rows], lr,
                      what=f"flashprefill_32k head {h}")
+
+
+@pytest.mark.parametrize("N,d,Hq,Hkv,alpha", [(3000, 128, 8, 2, 0.3), (2100, 64, 2, 2, 0.15)])
+def test_block_select_fp32_inputs(N, d, Hq, Hkv, alpha, cuda_device):
+    # fp32 Q/K (off the bf16 grid) through the same selection; the oracle
+    # reads the same fp32 values
+    from vs_workloads import bf16_bits_to_f32
+    Qb, Kb, _ = gen_qkv(N + 11, N, Hq, Hkv, d, 10000.0)
+    Qb, Kb = plant_block_structure(Qb, Kb, seed=N + 11)
+    rng = np.random.default_rng(N)
+    Qf = (bf16_bits_to_f32(Qb) * (1 + 1e-3 * rng.standard_normal(Qb.shape))).astype(np.float32)
+    Kf = (bf16_bits_to_f32(Kb) * (1 + 1e-3 * rng.standard_normal(Kb.shape))).astype(np.float32)
+    ref, margin = oracle.block_select(Qf, Kf, alpha)
+    assert (margin > 1e-9).all(), margin
+    got = _gpu_mask(torch.from_numpy(Qf).cuda(), torch.from_numpy(Kf).cuda(), alpha)
+    assert np.array_equal(got, ref)
