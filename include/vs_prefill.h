@@ -337,6 +337,15 @@ vs_status vs_read_device_status(const void* ws, cudaStream_t stream, int* flags)
  */
 vs_status vs_selftest_wait_timeout(void* ws, uint64_t limit_ns, cudaStream_t stream);
 
+/*
+ * Self-test of the fp64 exponential the block discovery uses for e^x, x <= 0
+ * (Tang's table-driven method; arguments below -700 give 0): y[i] = e^x[i]
+ * for the n device doubles at x (each <= 0 or -inf), written to the device
+ * array y.  Asynchronous on `stream`.  VS_ERR_INVALID_ARG for null pointers
+ * or n < 1.
+ */
+vs_status vs_selftest_exp(const double* x, double* y, int n, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

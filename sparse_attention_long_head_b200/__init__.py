@@ -43,7 +43,7 @@ EXPORTS = (
     "vs_selftest_wait_timeout", "vs_sparse_attn_fwd_static_scratch", "vs_attn_workspace_size_ld",
     "vs_attn_aggregate", "vs_attn_workspace_size_varlen", "vs_sparse_attn_fwd_varlen",
     "vs_dense_attn_fwd_varlen", "vs_block_select_workspace_size", "vs_block_select",
-    "vs_block_attn_workspace_size", "vs_block_sparse_attn_fwd",
+    "vs_block_attn_workspace_size", "vs_block_sparse_attn_fwd", "vs_selftest_exp",
 )
 
 
@@ -109,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.vs_read_device_status.restype = I
         L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
         L.vs_selftest_wait_timeout.restype = I
+        L.vs_selftest_exp.argtypes = [P, P, I, P]
+        L.vs_selftest_exp.restype = I
         L.vs_sparse_attn_fwd_static_scratch.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, I, P,
                                                         I64, P, P, I64, P, P, P, P]
         L.vs_sparse_attn_fwd_static_scratch.restype = I
@@ -300,6 +302,10 @@ def vs_read_device_status(ws, stream=None) -> tuple[int, int]:
 def vs_selftest_wait_timeout(ws, limit_ns: int, stream=None):
     _check(lib().vs_selftest_wait_timeout(_ptr(ws), int(limit_ns), _stream(stream)),
            "vs_selftest_wait_timeout")
+
+
+def vs_selftest_exp(x, y, stream=None):
+    _check(lib().vs_selftest_exp(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "vs_selftest_exp")
 
 
 # ------------------------------------------------------- allocation helpers

@@ -403,4 +403,9 @@ vs_status vs_selftest_wait_timeout(void* ws, uint64_t limit_ns, cudaStream_t str
   return launch_wait_selftest(status, limit_ns, stream) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
 }
 
+vs_status vs_selftest_exp(const double* x, double* y, int n, cudaStream_t stream) {
+  if (!x || !y || n < 1) return VS_ERR_INVALID_ARG;
+  return launch_exp_selftest(x, y, n, stream) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -82,6 +82,44 @@ __device__ __forceinline__ void dmma_16816(double (&c)[4], const double (&a)[8],
         "d"(b[0]), "d"(b[1]), "d"(b[2]), "d"(b[3]));
 }
 
+// e^x for x <= 0, branch-free, after Tang's table-driven method (P. T. P.
+// Tang, "Table-driven implementation of the exponential function in IEEE
+// floating-point arithmetic", ACM TOMS 15(2), 1989): x = (32 k + j) ln2/32 +
+// r with |r| <= ln2/64 (r from a two-constant reduction; n ln2/32 of the
+// high constant is exact for |n| < 2^17), e^r by its degree-5 Taylor
+// polynomial (truncation below 2e-15 relative), times tab[j] = 2^(j/32),
+// times 2^k by an exponent add.  Arguments below -700 (e^-700 < 1e-304,
+// negligible against the sums of at least 1 it feeds) and -inf give 0.
+constexpr double kExpInvStep = 46.16624130844683;       // 32 / ln 2
+constexpr double kExpStepHi = 0.021660849392446835;     // ln 2 / 32, 36 significant bits
+constexpr double kExpStepLo = 5.145609244655338e-14;    // ln 2 / 32 - kExpStepHi
+__device__ __forceinline__ double exp_nonpos(double x, const double* tab) {
+  const double xc = fmax(x, -700.0);
+  const double nd = rint(xc * kExpInvStep);
+  const int n = (int)nd;
+  const double r = fma(nd, -kExpStepLo, fma(nd, -kExpStepHi, xc));
+  double p = fma(r, 1.0 / 120.0, 1.0 / 24.0);
+  p = fma(r, p, 1.0 / 6.0);
+  p = fma(r, p, 0.5);
+  p = fma(r, p, 1.0);
+  p = fma(r, p, 1.0);
+  const double v = tab[n & 31] * p;  // in [2^-1/64, 2^(31/32 + 1/64)): exponent field 1022..1023
+  const double e = __hiloint2double(__double2hiint(v) + ((n >> 5) << 20), __double2loint(v));
+  return x >= -700.0 ? e : 0.0;
+}
+
+__device__ __forceinline__ void exp_table_init(double* tab) {
+  for (int j = threadIdx.x; j < 32; j += blockDim.x) tab[j] = exp2((double)j / 32.0);
+}
+
+__global__ void exp_selftest_kernel(const double* x, double* y, int n) {
+  __shared__ double tab[32];
+  exp_table_init(tab);
+  __syncthreads();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    y[i] = exp_nonpos(x[i], tab);
+}
+
 // Operand layout of the block means, per KV head g: tiles of 16 blocks, and
 // per tile D / 16 k-steps of 16 dimensions; a k-step is 4 x [32 lanes][2]
 // doubles, entry (j, lane = 4 r + t, e) holding kbar[16 tile + r + 8 e][16 ks
@@ -166,6 +204,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
   __shared__ double red[kBsWarps][4];
   __shared__ int item_slot;
   __shared__ int abort_flag;
+  __shared__ double exp_tab[32];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -178,6 +217,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
     abort_flag = 0;
     fence_mbar_init();
   }
+  exp_table_init(exp_tab);
   __syncthreads();
   const WaitCtx wc{a.wait_limit_ns, a.status, &abort_flag};
   const int esz = a.dtype == VS_BF16 ? 2 : 4;
@@ -440,10 +480,10 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
       double z0 = 0.0, z1 = 0.0;
       sweep(true, [&](int q, int m, double (&v)[4]) {
         const int J0 = 16 * (kTilesPerStage * q + m) + gq, J1 = J0 + 8;
-        v[0] = pv0 && J0 < I ? exp(v[0] - pm0) : 0.0;
-        v[1] = pv1 && J0 < I ? exp(v[1] - pm1) : 0.0;
-        v[2] = pv0 && J1 < I ? exp(v[2] - pm0) : 0.0;
-        v[3] = pv1 && J1 < I ? exp(v[3] - pm1) : 0.0;
+        v[0] = pv0 && J0 < I ? exp_nonpos(v[0] - pm0, exp_tab) : 0.0;
+        v[1] = pv1 && J0 < I ? exp_nonpos(v[1] - pm1, exp_tab) : 0.0;
+        v[2] = pv0 && J1 < I ? exp_nonpos(v[2] - pm0, exp_tab) : 0.0;
+        v[3] = pv1 && J1 < I ? exp_nonpos(v[3] - pm1, exp_tab) : 0.0;
         z0 += v[0] + v[2];
         z1 += v[1] + v[3];
       });
@@ -527,6 +567,11 @@ int num_sms() {
 int64_t scratch_doubles_per_cta(int Tp) { return (int64_t)(Tp / (16 * kTilesPerStage)) * 8 * 256; }
 
 }  // namespace
+
+cudaError_t launch_exp_selftest(const double* x, double* y, int n, cudaStream_t stream) {
+  exp_selftest_kernel<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 size_t block_select_ws_bytes(int N, int Hkv, int d) {
   const int T = (N + 127) / 128, Tp = pad_blocks(T), sms = num_sms();

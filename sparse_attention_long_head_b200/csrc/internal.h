@@ -215,6 +215,7 @@ struct BlockSelectArgs {
 };
 size_t block_select_ws_bytes(int N, int Hkv, int d);
 cudaError_t launch_block_select(const BlockSelectArgs& a);
+cudaError_t launch_exp_selftest(const double* x, double* y, int n, cudaStream_t stream);
 
 // Launchers (return a CUDA error; argument checks are done by the caller).
 cudaError_t launch_plan(const AttnArgs& a, const PlanLayout& L);

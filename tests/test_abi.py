@@ -201,6 +201,8 @@ def test_indexer_and_misc_host_validation():
     assert L.vs_read_device_status(None, None, ctypes.byref(flags)) == vs.VS_ERR_INVALID_ARG
     assert L.vs_selftest_wait_timeout(None, 1000000, None) == vs.VS_ERR_WORKSPACE
     assert L.vs_selftest_wait_timeout(f(0x10000), 10, None) == vs.VS_ERR_INVALID_ARG
+    assert L.vs_selftest_exp(None, f(0x10000), 4, None) == vs.VS_ERR_INVALID_ARG
+    assert L.vs_selftest_exp(f(0x10000), f(0x20000), 0, None) == vs.VS_ERR_INVALID_ARG
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):
