@@ -1123,10 +1123,34 @@ def run_blocks(args, w):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = block_oracle_sample(w, Qb, Kb, Vb, mask_h, args.cpu_seconds)
     out["clocks"] = clk.summary()
+    out["kernels"] = block_kernel_rooflines(N, Hq, d, ms_step - ms_att, ms_att, flops, t_roof_ms,
+                                            out["clocks"], torch.cuda.get_device_properties(dev))
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+FP64_FMA_PER_CLK_SM = 64  # fp64 FMA (vector or mma.sync) per clock per SM, measured on the B200
+
+
+def block_kernel_rooflines(N, Hq, d, ms_disc, ms_att, att_flops, att_roof_ms, clocks, props):
+    """Discovery against its fp64 bound: 16 probes x d FMA per (head, query
+    block I, key block J < I); the peak is SMs x 64 fp64 FMA/clk x the SM
+    clock sampled during the run.  Attention as in the main roofline."""
+    T = (N + 127) // 128
+    fma = 16.0 * d * Hq * T * (T - 1) / 2
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    peak = props.multi_processor_count * FP64_FMA_PER_CLK_SM * 2 * mhz * 1e6 / 1e12
+    achieved = 2 * fma / (ms_disc * 1e-3) / 1e12
+    return {
+        "discovery": {"ms": round(ms_disc, 3), "bound": "fp64", "achieved_tflops": round(achieved, 2),
+                      "peak_tflops": round(peak, 2), "frac": round(achieved / peak, 4),
+                      "peak_source": "SMs x 64 fp64 FMA/clk/SM (measured) x sampled SM clock"},
+        "attention": {"ms": round(ms_att, 3), "bound": "tensor",
+                      "achieved_tflops": round(att_flops / (ms_att * 1e-3) / 1e12, 2),
+                      "frac": round(att_roof_ms / ms_att, 4)},
+    }
 
 
 def block_oracle_sample(w, Qb, Kb, Vb, mask, seconds, seed=0,

@@ -45,3 +45,19 @@ def test_block_pairs_brute_force():
                 for j in range(i + 1):
                     want += int(keep[h, i // 128, j // 128])
         assert bench.block_pairs(mask, N) == want
+
+
+def test_block_kernel_rooflines():
+    import types
+    props = types.SimpleNamespace(multi_processor_count=148)
+    k = bench.block_kernel_rooflines(131072, 32, 128, 4.0, 8.0, 1e15, 6.0,
+                                     {"sm_mhz": 1965.0}, props)
+    T = 1024
+    fma = 16 * 128 * 32 * T * (T - 1) / 2
+    peak = 148 * 64 * 2 * 1965e6 / 1e12
+    assert abs(k["discovery"]["achieved_tflops"] - round(2 * fma / 4e-3 / 1e12, 2)) < 1e-9
+    assert abs(k["discovery"]["peak_tflops"] - round(peak, 2)) < 1e-9
+    assert k["attention"]["frac"] == 0.75
+    # no clock samples: the nominal maximum clock
+    k2 = bench.block_kernel_rooflines(131072, 32, 128, 4.0, 8.0, 1e15, 6.0, {"sm_mhz": None}, props)
+    assert k2["discovery"]["peak_tflops"] == k["discovery"]["peak_tflops"]
