@@ -261,8 +261,10 @@ cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L) {
 
 // For each (head h, pair p) of query blocks I = 2p, 2p + 1: the ascending
 // union of the key blocks kept for either (J <= I each), with bit 30 / 31
-// marking the blocks kept for the first / second.  One warp per unit; the
-// rows have at most 64 words (T <= 2048).
+// marking the blocks kept for the first / second, and bit 28 / 29 the last
+// block kept for the first / second (the attention then knows when a
+// sub-tile's accumulation is complete).  One warp per unit; the rows have at
+// most 64 words (T <= 2048).
 __global__ void __launch_bounds__(32) block_plan_kernel(const uint32_t* mask, int T, int P,
                                                         int32_t* bcnt, uint32_t* blist) {
   const int p = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
@@ -299,6 +301,14 @@ __global__ void __launch_bounds__(32) block_plan_kernel(const uint32_t* mask, in
       out[pos++] = J | (((a >> bit) & 1u) << 30) | (((b >> bit) & 1u) << 31);
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  if (lane < 2) {  // lane s marks the last entry kept for sub-tile s
+    for (int k = base - 1; k >= 0; --k)
+      if ((out[k] >> (30 + lane)) & 1u) {
+        atomicOr(&out[k], 1u << (28 + lane));
+        break;
+      }
   }
   if (lane == 0) bcnt[(int64_t)h * P + p] = base;
 }
@@ -428,7 +438,8 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
 struct Item {
   int kind;
   int b;      // key block (tile) or chunk index (vertical chunk)
-  int flags;  // block sparse: bit s set iff the block is kept for sub-tile s
+  int flags;  // block sparse: bit s set iff the block is kept for sub-tile s,
+              // bit 2 + s iff it is the last block kept for sub-tile s
 };
 
 __device__ __forceinline__ Item unit_item(const AttnParams& P, const UnitInfo& ui, int k) {
@@ -438,7 +449,7 @@ __device__ __forceinline__ Item unit_item(const AttnParams& P, const UnitInfo& u
     const uint32_t e = P.blist[(int64_t)ui.d1start + k];
     it.kind = kItemTile;
     it.b = (int)(e & 0xFFFFu);
-    it.flags = (int)(e >> 30);
+    it.flags = (int)((e >> 30) | (((e >> 28) & 3u) << 2));
   } else if (ui.mode != kModeSplit) {
     it.kind = kItemTile;
     it.b = k;
@@ -483,7 +494,7 @@ __device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& u
   const int b = it.b;
   // causal part for the keys of block b: keep c <= i - 128 b
   const bool below = b < t_sub;  // whole block in the past of every row of the sub-tile
-  if (MODE == kAttnBlock && !((it.flags >> (t_sub - 2 * ui.p)) & 1)) {
+  if (MODE == kAttnBlock && !((it.flags >> (t_sub - 2 * ui.p)) & 1)) {  // (callers skip these)
 #pragma unroll
     for (int q = 0; q < 4; ++q) w[q] = 0u;  // not kept for this sub-tile's query block
     return true;
@@ -684,8 +695,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         continue;
       }
       float m_use = -INFINITY, l = 0.f;
+      int nproc = 0;  // items this sub-tile has processed
       for (int k = 0; k < ui.n; ++k) {
         const Item it = unit_item(P, ui, k);
+        // block sparse: the MMA issuer gives this sub-tile only the blocks it keeps
+        if (MODE == kAttnBlock && !((it.flags >> sub) & 1)) continue;
         uint32_t mw[4];
         const bool masked = item_mask<MODE>(P, ui, it, im, t_sub, mw);
         if (!mbar_wait(bar(B_SFULL + sub), scnt & 1, wc)) { ok = false; break; }
@@ -729,9 +743,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float ls = 0.f;
         exp_tile(sr, mw, masked, P.scale_log2, m_base, tS, ls);
         l += ls;
-        if (k > 0 && __any_sync(0xffffffffu, need)) {
-          // O must be rescaled before PV(k) accumulates into it; PV(k-1) is
-          // complete because S(k) was issued after it.
+        if (nproc > 0 && __any_sync(0xffffffffu, need)) {
+          // O must be rescaled before PV(k) accumulates into it; the previous
+          // PV is complete because S(k) was issued after it.
 #pragma unroll 1
           for (int q = 0; q < D / 32; ++q) {
             uint32_t o[32];
@@ -745,17 +759,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL + sub));
+        ++nproc;
       }
       if (!ok) break;
       if (!mbar_wait(bar(B_OFULL + sub), ucount & 1, wc)) { ok = false; break; }
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      // no key at all (block sparse: possibly no PV, so O holds stale values)
+      const bool empty_row = MODE == kAttnBlock && !(l > 0.f);
       __nv_bfloat16* orow = orow_of();
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * q, o);
         tmem_ld_wait(o);
+        if (empty_row) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
         if (i < ui.Nb) {
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
@@ -808,6 +829,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const UnitInfo ui = unit_info<MODE>(P, u);
         if (ui.n == 0) continue;
         if (!mbar_wait(bar(B_QFULL), ucount & 1, wc)) { ok = false; break; }
+        if constexpr (MODE == kAttnBlock) {
+          // Each sub-tile gets S and PV only for the blocks it keeps; K and V
+          // of every listed block stream through the ring as in the other
+          // modes.  At the stage [V(k), K(k+1)]: PV(k) for the sub-tiles
+          // keeping block k (O complete after a sub-tile's last one), then
+          // S(k+1) for those keeping block k+1 -- after the sub-tile's
+          // previous PV in issue order, so S never overwrites an unread P.
+          int fl = unit_item(P, ui, 0).flags;
+          int fl_next = ui.n > 1 ? unit_item(P, ui, 1).flags : 0;
+          bool started[2] = {false, false};
+          uint32_t kslot = seq % S;
+          if (!mbar_wait(bar(B_STAGE + stg % S), (stg / S) & 1, wc)) { ok = false; break; }  // [K(0)]
+          ++seq;
+          ++stg;
+          tc_fence_after();
+          for (int sub = 0; sub < 2; ++sub)
+            if ((fl >> sub) & 1) {
+              issue_s(sub, kslot);
+              mma_commit(bar(B_SFULL + sub));
+            }
+          mma_commit(bar(B_EMPTY + kslot));
+          for (int k = 0; k < ui.n && ok; ++k) {
+            const int fl_after = k + 2 < ui.n ? unit_item(P, ui, k + 2).flags : 0;  // early load
+            if (!mbar_wait(bar(B_STAGE + stg % S), (stg / S) & 1, wc)) { ok = false; break; }
+            ++stg;
+            const uint32_t vslot = seq % S;
+            ++seq;
+            if (k + 1 < ui.n) {
+              kslot = seq % S;
+              ++seq;
+            }
+            for (int sub = 0; sub < 2; ++sub) {
+              if ((fl >> sub) & 1) {
+                if (!mbar_wait(bar(B_PFULL + sub), pcnt[sub] & 1, wc)) { ok = false; break; }
+                ++pcnt[sub];
+                tc_fence_after();
+                issue_pv(sub, vslot, started[sub]);
+                started[sub] = true;
+                if ((fl >> (2 + sub)) & 1) mma_commit(bar(B_OFULL + sub));
+              }
+              if (k + 1 < ui.n && ((fl_next >> sub) & 1)) {
+                issue_s(sub, kslot);
+                mma_commit(bar(B_SFULL + sub));
+              }
+            }
+            if (!ok) break;
+            mma_commit(bar(B_EMPTY + vslot));
+            if (k + 1 < ui.n) mma_commit(bar(B_EMPTY + kslot));
+            fl = fl_next;
+            fl_next = fl_after;
+          }
+          if (!ok) break;
+          // a sub-tile without kept blocks (rows past the sequence's end, or an
+          // empty mask row): its epilogue writes zeros from l = 0
+          for (int sub = 0; sub < 2; ++sub)
+            if (!started[sub]) mma_commit(bar(B_OFULL + sub));
+          mma_commit(bar(B_QEMPTY));
+          ++ucount;
+          continue;
+        }
         uint32_t kslot = seq % S;
         if (!mbar_wait(bar(B_STAGE + stg % S), (stg / S) & 1, wc)) { ok = false; break; }  // [K(0)]
         ++seq;

@@ -183,3 +183,28 @@ def test_block_select_fp32_inputs(N, d, Hq, Hkv, alpha, cuda_device):
     assert (margin > 1e-9).all(), margin
     got = _gpu_mask(torch.from_numpy(Qf).cuda(), torch.from_numpy(Kf).cuda(), alpha)
     assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("N,d,Hq,Hkv,dens,seed", [(2049, 128, 2, 1, 0.15, 1), (1500, 64, 2, 2, 0.5, 2),
+                                                  (3000, 128, 4, 2, 0.05, 3)])
+def test_random_masks_per_sub_tile(N, d, Hq, Hkv, dens, seed, cuda_device):
+    # each query block keeps its own random set (the two query blocks of a
+    # pair differ; some drop their diagonal; one keeps nothing)
+    Qb, Kb, Vb = gen_qkv(seed + 30, N, Hq, Hkv, d, 10000.0)
+    T = (N + 127) // 128
+    W = (T + 31) // 32
+    rng = np.random.default_rng(seed)
+    bits = rng.random((Hq, T, T)) < dens
+    bits |= np.eye(T, dtype=bool)[None] & (rng.random((Hq, T, 1)) < 0.8)
+    bits[0, T // 2, :] = False
+    mask = np.zeros((Hq, T, W), np.uint32)
+    for J in range(T):
+        mask[:, :, J // 32] |= (bits[:, :, J].astype(np.uint32) << np.uint32(J % 32))
+    O, lse = _gpu_block_attn(Qb, Kb, Vb, mask)
+    Od = dev_to_f64(O)
+    lsed = lse.cpu().numpy().astype(np.float64)
+    for h in range(Hq):
+        Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, np.arange(N), mask)
+        compare_rows(Od[:, h], Or, lsed[h], lr, what=f"head {h}")
+    r0 = 128 * (T // 2)
+    assert np.all(Od[r0:r0 + 128, 0] == 0) and np.all(np.isneginf(lsed[0, r0:r0 + 128]))
