@@ -96,7 +96,8 @@ def test_full_size_workload(name, cuda_device):
 
     Od = dev_to_f64(O)
     lsed = lse.cpu().numpy().astype(np.float64)
-    n_random = 256 if N <= 32768 else 96
+    # 4096 seeded random rows per head (1024 at 256K, where a row has ~32K keys)
+    n_random = 4096 if N <= 131072 else 1024
     worst = 0.0
     for h in range(Hq):
         hs = h * w.H_sel // Hq
