@@ -21,15 +21,16 @@
 //     probes per MMA n-tile) heaviest first from a counter.  The dot products
 //     are mma.sync m16n8k16 fp64 (16 key blocks x 8 probes x 16 dims per
 //     instruction: one instruction where vector code needs 64, at the same
-//     fp64 rate).  Each consumer warp keeps its n-tile's probe fragments in
-//     registers; a producer warp streams the block means through a ring of
-//     shared-memory stages (two 16-block tiles each) with bulk copies, and
-//     every tile of a stage feeds all the item's n-tiles.
-//     Pass 1: the dot products, each probe's online maximum and sum of
-//     exponentials, and the dot products stored in the CTA's scratch.
-//     Pass 2: from the scratch, each probe's normalised exponentials summed
-//     over the head's 16 probes give the block scores in shared memory;
-//     then the maximum, the threshold and the row's bitmask.
+//     fp64 rate).  A producer warp stages each item's probes as fp64 MMA
+//     B-fragments in shared memory and streams the block means through a
+//     ring of shared-memory stages (two 16-block tiles each) with bulk
+//     copies; every tile of a stage feeds all the item's n-tiles.  Eight
+//     consumer warps then run three passes per item:
+//     pass 1: the dot products (stored in the CTA's scratch) and each
+//       probe's maximum;
+//     pass 2: e = exp(s - max) back into the scratch, and the sums Z;
+//     pass 3: the block scores sum_p e / Z_p in shared memory, then each
+//       head's maximum, threshold and bitmask row.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -170,7 +171,7 @@ struct ScoreArgs {
 
 // Persistent: one CTA per SM; work items are (query block I, chunk of HC
 // query heads), heaviest rows first, claimed from a global counter by the
-// producer warp, which also stages each item's probe rows (raw input type)
+// producer warp, which also stages each item's probes as fp64 B-fragments
 // and streams its block means through the ring, so the next item's data
 // arrives while the consumers finish the current one.  Per item the eight
 // consumer warps run:
@@ -630,8 +631,8 @@ cudaError_t launch_block_select(const BlockSelectArgs& a) {
   if (dyn_bytes(s.stages) > kMaxDynSmem) s.stages = 2;
   const size_t need = dyn_bytes(s.stages);
   if (need > kMaxDynSmem) return cudaErrorInvalidValue;
-  // more than half of an SM's shared memory: one CTA per SM, so a CTA's
-  // scratch slot (its block index) is never shared
+  // more than half of an SM's shared memory: the persistent grid (one CTA
+  // per SM) cannot pile two CTAs onto one SM while another stays idle
   const size_t smem = need > kOneCtaSmem ? need : kOneCtaSmem;
   auto kern = a.d == 128 ? (HC == 4 ? block_score_kernel<128, 2> : block_score_kernel<128, 1>)
                          : (HC == 4 ? block_score_kernel<64, 2> : block_score_kernel<64, 1>);
