@@ -613,7 +613,11 @@ def run_ours(args, w):
                      "kernel": "vs_sparse_attn_fwd (plan + attn_tc_kernel)",
                      "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)",
                      "frac_vs_burst_peak": round(flops / (peaks["bf16_tflops"] * 1e12) * 1e3 / ms_att, 4),
-                     "t_roof_ms": round(t_roof_ms, 3)},
+                     "t_roof_ms": round(t_roof_ms, 3),
+                     # the HBM term against the measured copy rate and the nominal ~8 TB/s
+                     "hbm_bytes": int(algo_bytes),
+                     "hbm_frac_measured": round(algo_bytes / (peaks["hbm_gbs"] * 1e9) / (ms_att * 1e-3), 5),
+                     "hbm_frac_nominal_8tbs": round(algo_bytes / 8e12 / (ms_att * 1e-3), 5)},
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "input_gen_s": round(gen_s, 1),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -720,11 +724,21 @@ def cpu_baseline(w, Qb, Kb, Vb, vi, vc, si, sc, seconds, seed=0,
         pairs += int(row_pairs(rows, vi[hs, : vc[hs]], si[hs, : sc[hs]]).sum())
         rows_done += rows.size
         heads.append(h)
+    # the dense causal oracle per row, likewise (a few rows spread over the sequence)
+    drows = np.sort(rng.integers(N // 2, N, 16))
+    t0 = time.time()
+    oracle.attn_rows(Qb, Kb, Vb, 0, drows, dense=True)
+    dense_row_ms = (time.time() - t0) * 1e3 / drows.size
+    dense_pairs_per_row = float(np.mean(drows + 1))
     return {"value": round(4.0 * d * pairs / t_used / 1e12, 6), "unit": UNIT, "cores": _cpu_cores(),
             "kind": "oracle",
             "sample": f"{rows_done} query rows (32 random rows of a random head per draw, "
                       f"{len(set(heads))} heads) of {w.name}, fp64 row-form oracle with OpenMP over "
-                      f"rows, {t_used:.1f} s; index sets from {sets_from}"}
+                      f"rows, {t_used:.1f} s; index sets from {sets_from}",
+            "sparse_row_ms": round(t_used * 1e3 / max(rows_done, 1), 4),
+            "dense_row_ms": round(dense_row_ms, 4),
+            "dense_row_sample": f"16 random rows of the second half, head 0, "
+                                f"{dense_pairs_per_row:.0f} keys per row on average"}
 
 
 def run_reference(args, w):

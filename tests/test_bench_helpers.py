@@ -61,3 +61,21 @@ def test_block_kernel_rooflines():
     # no clock samples: the nominal maximum clock
     k2 = bench.block_kernel_rooflines(131072, 32, 128, 4.0, 8.0, 1e15, 6.0, {"sm_mhz": None}, props)
     assert k2["discovery"]["peak_tflops"] == k["discovery"]["peak_tflops"]
+
+
+def test_cpu_baseline_reports_sparse_and_dense_rows():
+    import oracle
+    from vs_workloads import WORKLOADS
+    w = WORKLOADS["tiny_1k"]
+    Qb, Kb, Vb = w.qkv()
+    lv, ls = w.all_scores()
+    sets = []
+    for scores, k, tau in ((lv, w.k_v, w.tau_v), (ls, w.k_s, w.tau_s)):
+        idx = np.empty((w.H_sel, k), np.int32)
+        cnt = np.empty(w.H_sel, np.int32)
+        for h in range(w.H_sel):
+            idx[h], cnt[h], _ = oracle.select(scores[h], w.select_mode_id, k, tau)
+        sets += [idx, cnt]
+    cb = bench.cpu_baseline(w, Qb, Kb, Vb, *sets, seconds=0.05)
+    assert cb["kind"] == "oracle" and cb["value"] > 0
+    assert cb["sparse_row_ms"] > 0 and cb["dense_row_ms"] > 0
