@@ -57,3 +57,24 @@ def test_indexer_workload_then_select(cuda_device):
     ties = check_select(lv.astype(np.float32), vs.VS_SELECT_THRESHOLD, w.k_v, w.tau_v)
     ties += check_select(ls.astype(np.float32), vs.VS_SELECT_THRESHOLD, w.k_s, w.tau_s)
     assert ties == []
+
+
+@pytest.mark.parametrize("d,pad", [(40, 0), (128, 3)])
+def test_general_layout_path(d, pad, cuda_device):
+    # d not a multiple of 16, or a token stride off the 16-byte grid: the
+    # kernel for arbitrary strides
+    N, Hkv, hidden = 300, 2, 256
+    _, Kb, Vb = gen_qkv(d + pad, N, Hkv, Hkv, d, 500000.0)
+    rng = np.random.default_rng(d)
+    W1 = (0.02 * rng.standard_normal((hidden, 2 * d))).astype(np.float32)
+    W2 = (0.02 * rng.standard_normal((2, hidden))).astype(np.float32)
+
+    def padded(bits):
+        buf = torch.zeros((N, Hkv * d + pad), dtype=torch.int16)
+        buf[:, : Hkv * d] = torch.from_numpy(bits.reshape(N, Hkv * d).view(np.int16))
+        return buf.cuda().view(torch.bfloat16)[:, : Hkv * d].view(N, Hkv, d) if pad == 0 else \
+            buf.cuda().view(torch.bfloat16).as_strided((N, Hkv, d), (Hkv * d + pad, d, 1))
+
+    lv, ls = _run(padded(Kb), padded(Vb), W1, W2)
+    rv, rs = oracle.index_scores(Kb, Vb, W1, W2)
+    assert np.abs(lv - rv).max() <= TOL and np.abs(ls - rs).max() <= TOL
