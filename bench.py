@@ -633,9 +633,10 @@ def kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, att_bytes, ms_att, m
                      ld_v, ld_s, agg=None):
     """Per hot-path kernel: achieved vs the roofline that bounds it.
     attention (+plan, +pack): tensor-bound, 4 d P flops; select x2: HBM-bound,
-    4 B per score read + 4 B per index slot written; indexer: fp32 CUDA-core
-    FMA-bound, 2 (2d hidden + 2 hidden) flops per (token, KV head), peak =
-    148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz."""
+    4 B per score read + 4 B per index slot written; indexer (bf16 rows, the
+    tensor-core kernel): 2 (2d hidden + 2 hidden) flops and 2 x 2d bytes of
+    [k; v] in plus 8 B of logits out per (token, KV head), bound by the slower
+    of the bf16 tensor peak (burst: the kernel is timed alone) and HBM."""
     out = {}
     peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     t_att = flops / (peak_t * 1e12)
@@ -658,11 +659,14 @@ def kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, att_bytes, ms_att, m
     if w.indexer:
         hidden = w.hidden
         iflops = 2.0 * N * Hkv * (2 * d * hidden + 2 * hidden)
-        alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6
-        out["indexer"] = {"ms": round(ms_idx, 3), "bound": "alu",
+        ibytes = N * Hkv * (2.0 * 2 * d + 8.0) + 4.0 * hidden * (2 * d + 2)
+        t_tc = iflops / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = ibytes / (peaks["hbm_gbs"] * 1e9)
+        out["indexer"] = {"ms": round(ms_idx, 3), "bound": "tensor" if t_tc >= t_hbm else "hbm",
                           "achieved_tflops": round(iflops / (ms_idx * 1e-3) / 1e12, 2),
-                          "peak_tflops": round(alu_peak / 1e12, 1),
-                          "frac": round(iflops / alu_peak / (ms_idx * 1e-3), 4)}
+                          "achieved_gbs": round(ibytes / (ms_idx * 1e-3) / 1e9, 1),
+                          "t_roof_ms": round(max(t_tc, t_hbm) * 1e3, 4),
+                          "frac": round(max(t_tc, t_hbm) / (ms_idx * 1e-3), 4)}
     return out
 
 

@@ -9,12 +9,26 @@
 // the 16 threads that share a row with warp shuffles.  Hidden sizes above
 // 256 loop over 256-wide slices and accumulate the two outputs.
 //
+// index_scores_tc_kernel (bf16 inputs, d = 64 or 128, hidden = 128 or 256,
+// heads contiguous in a token row, 16-byte aligned rows) runs X W1^T on the
+// tensor cores: W1 = hi + lo with hi = bf16(W1) and lo = bf16(W1 - hi)
+// (residual below 2^-17 of |W1|), and X W1^T = X hi^T + X lo^T as two bf16
+// MMAs with fp32 accumulation (bf16 x bf16 products are exact in fp32).  Persistent CTAs
+// each keep one 128-unit hidden slice of both parts in shared memory (128-
+// byte-swizzled, K-major), stage a 128-token X tile per step with 16-byte
+// loads, and accumulate the 128 x 128 tile in TMEM; the epilogue applies ReLU
+// and the slice's share of the down-projection and adds it to the logits
+// (zeroed first; at most two slices, so the order of the two additions does
+// not change the sum).  A device wait that runs out (a correct launch never
+// does) leaves NaN in the logits of that tile and of the CTA's later tiles.
+//
 // index_scores_vec_kernel is the same computation for aligned inputs (16-byte
 // aligned rows, d a multiple of 16): a CTA takes 128 consecutive tokens of
 // one KV head, so its X rows are contiguous and load as 16-byte vectors, W1
 // loads as float4, and the next K-chunk is in registers while the current
 // one is multiplied.
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace vs {
 
@@ -260,6 +274,133 @@ __global__ void __launch_bounds__(kIdxThreads) index_scores_vec_kernel(IdxArgs a
   }
 }
 
+constexpr int kTcThreads = 128;
+constexpr uint64_t kTcWaitNs = kDefaultWaitLimitNs;
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1) index_scores_tc_kernel(IdxArgs a, int slices) {
+  constexpr int KB = 2 * D / 64;       // 64-feature boxes of one [k; v] row
+  constexpr int kBox = 128 * 128;      // bytes of a 128-row x 64-bf16 box
+  extern __shared__ uint8_t dyn_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sW = smem;                  // [2 parts][KB boxes]
+  uint8_t* sX = smem + 2 * KB * kBox;  // [KB boxes]
+  __shared__ float w2s[2][128];
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int j = blockIdx.x % slices;   // hidden slice [128 j, 128 j + 128)
+  const int D2 = 2 * D;
+  // W1 slice -> hi / lo bf16 parts, 8 features (one 16-byte chunk) at a time
+  for (int e = tid; e < 128 * (D2 / 8); e += kTcThreads) {
+    const int n = e / (D2 / 8), c = (e % (D2 / 8)) * 8;
+    const float4* src = reinterpret_cast<const float4*>(a.W1 + (int64_t)(128 * j + n) * D2 + c);
+    const float4 f0 = __ldg(src), f1 = __ldg(src + 1);
+    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(f[2 * y]), h1 = __float2bfloat16_rn(f[2 * y + 1]);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(f[2 * y] - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(f[2 * y + 1] - __bfloat162float(h1));
+      hi[y] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      lo[y] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    const uint32_t off = (c / 64) * kBox + sw128_off(n, (c % 64) / 8);
+    *reinterpret_cast<uint4*>(sW + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(sW + KB * kBox + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  for (int e = tid; e < 256; e += kTcThreads) w2s[e / 128][e % 128] = a.W2[(e / 128) * a.hidden + 128 * j + e % 128];
+  if (tid == 0) {
+    mbar_init(smem_u32(&mma_bar), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tslot), 128);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tacc = tslot;
+  constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+  const uint64_t xdesc = sdesc_sw128(smem_u32(sX), 16, 1024);
+  const uint64_t wdesc = sdesc_sw128(smem_u32(sW), 16, 1024);
+  const int64_t ntile = (a.N + 127) / 128;
+  const int64_t items = ntile * a.Hkv;
+  const int per = gridDim.x / slices;  // CTAs per slice
+  uint32_t phase = 0;
+  bool dead = false;  // CTA-uniform: a wait for this CTA's MMAs ran out
+  for (int64_t it = blockIdx.x / slices; it < items; it += per) {
+    const int g = (int)(it % a.Hkv);
+    const int64_t t0 = (it / a.Hkv) * 128;
+    float pv = __int_as_float(0x7fc00000), ps = pv;  // NaN unless the tile completes
+    if (!dead) {
+      // X tile: 128 tokens x [k; v], 16-byte chunks into the swizzled boxes
+      for (int e = tid; e < 128 * (D2 / 8); e += kTcThreads) {
+        const int r = e / (D2 / 8), c = (e % (D2 / 8)) * 8;
+        const int64_t t = t0 + r;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (t < a.N) {
+          const uint16_t* base = static_cast<const uint16_t*>(c < D ? a.K : a.V);
+          v = __ldg(reinterpret_cast<const uint4*>(base + t * a.stride_tok + (int64_t)g * D + (c % D)));
+        }
+        *reinterpret_cast<uint4*>(sX + (c / 64) * kBox + sw128_off(r, (c % 64) / 8)) = v;
+      }
+      fence_proxy_async_smem();  // generic-proxy stores -> the tensor core's reads
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int kk = 0; kk < D2 / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+            mma_ss(tacc, xdesc + off, wdesc + ((p * KB * kBox) >> 4) + off, idesc,
+                   (p | kk) ? 1u : 0u);
+          }
+        mma_commit(smem_u32(&mma_bar));
+      }
+      // warp-uniform, since tcgen05.ld is a warp-wide instruction
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_drain(smem_u32(&mma_bar), phase, kTcWaitNs));
+      tc_fence_after();
+      if (ok) {
+        // epilogue: thread tid = token row; TMEM lanes 32 warp .. 32 warp + 31
+        pv = ps = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v[32];
+          tmem_ld32(tacc + ((uint32_t)(warp * 32) << 16) + 32 * q, v);
+          tmem_ld_wait(v);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float h = fmaxf(__uint_as_float(v[c]), 0.f);
+            pv = fmaf(w2s[0][32 * q + c], h, pv);
+            ps = fmaf(w2s[1][32 * q + c], h, ps);
+          }
+        }
+      }
+      tc_fence_before();
+      // TMEM and the X tile are reused by the next tile
+      dead = __syncthreads_or(!ok) != 0;
+      if (!dead) phase ^= 1u;
+    }
+    const int64_t t = t0 + tid;
+    if (t < a.N) {
+      atomicAdd(&a.lv[(int64_t)g * a.N + t], pv);
+      atomicAdd(&a.ls[(int64_t)g * a.N + t], ps);
+    }
+  }
+  // after a timeout, let the MMAs in flight land before TMEM is released
+  if (dead) mbar_wait_drain(smem_u32(&mma_bar), phase, kTcWaitNs);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tacc, 128);
+  }
+}
+
 cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, int Hkv, int d,
                                 int64_t stride_tok, int64_t stride_head, const float* W1,
                                 const float* W2, int hidden, float* lv, float* ls,
@@ -267,6 +408,34 @@ cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, 
   IdxArgs a{K, V, dtype, N, Hkv, d, stride_tok, stride_head, W1, W2, hidden, lv, ls};
   const int esz = dtype == VS_BF16 ? 2 : 4;
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  const bool tc = dtype == VS_BF16 && (d == 64 || d == 128) && (hidden == 128 || hidden == 256) &&
+                  stride_head == d && (stride_tok * 2) % 16 == 0 && al16(K) && al16(V) &&
+                  al16(W1);
+  if (tc) {
+    const int slices = hidden / 128;
+    const int kb = 2 * d / 64;
+    const size_t smem = (size_t)3 * kb * 128 * 128 + 1024;  // W1 hi / lo parts, X tile, alignment
+    if (cudaMemsetAsync(lv, 0, sizeof(float) * (size_t)N * Hkv, stream) != cudaSuccess ||
+        cudaMemsetAsync(ls, 0, sizeof(float) * (size_t)N * Hkv, stream) != cudaSuccess)
+      return cudaErrorUnknown;
+    const int64_t items = ((int64_t)N + 127) / 128 * Hkv;
+    int grid = device_sm_count() / slices * slices;
+    if ((int64_t)grid > items * slices) grid = (int)(items * slices);
+    if (grid < slices) grid = slices;
+    cudaError_t e;
+    if (d == 128) {
+      e = cudaFuncSetAttribute(index_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e != cudaSuccess) return e;
+      index_scores_tc_kernel<128><<<grid, kTcThreads, smem, stream>>>(a, slices);
+    } else {
+      e = cudaFuncSetAttribute(index_scores_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e != cudaSuccess) return e;
+      index_scores_tc_kernel<64><<<grid, kTcThreads, smem, stream>>>(a, slices);
+    }
+    return cudaGetLastError();
+  }
   const bool vec = d % kIdxK == 0 && (stride_tok * esz) % 16 == 0 && (stride_head * esz) % 16 == 0 &&
                    al16(K) && al16(V) && al16(W1) && (2 * d) % 4 == 0 && N <= (1 << 30);
   if (vec) {

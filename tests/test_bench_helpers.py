@@ -79,3 +79,17 @@ def test_cpu_baseline_reports_sparse_and_dense_rows():
     cb = bench.cpu_baseline(w, Qb, Kb, Vb, *sets, seconds=0.05)
     assert cb["kind"] == "oracle" and cb["value"] > 0
     assert cb["sparse_row_ms"] > 0 and cb["dense_row_ms"] > 0
+
+
+def test_indexer_roofline_terms():
+    import types
+    w = types.SimpleNamespace(indexer=True, hidden=256)
+    peaks = {"bf16_tflops": 1500.0, "hbm_gbs": 6000.0}
+    N, Hkv, d = 262144, 8, 128
+    k = bench.kernel_rooflines(w, peaks, N, 32, Hkv, d, 8, 1e15, 1e9, 10.0, 1.0, 2.0, 0, 0)
+    flops = 2.0 * N * Hkv * (2 * d * 256 + 2 * 256)
+    nbytes = N * Hkv * (4 * d + 8) + 4 * 256 * (2 * d + 2)
+    t = max(flops / 1.5e15, nbytes / 6e12)
+    assert k["indexer"]["bound"] == ("tensor" if flops / 1.5e15 >= nbytes / 6e12 else "hbm")
+    assert abs(k["indexer"]["frac"] - round(t / 2e-3, 4)) < 1e-12
+    assert abs(k["indexer"]["achieved_gbs"] - round(nbytes / 2e-3 / 1e9, 1)) < 1e-9

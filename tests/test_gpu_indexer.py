@@ -1,5 +1,8 @@
-"""vs_index_scores on the GPU vs the fp64 oracle: max-abs <= 1e-5 (fp32
-CUDA-core arithmetic, logits of std ~0.06 at the 0.02-std weights)."""
+"""vs_index_scores on the GPU vs the fp64 oracle: max-abs <= 1e-5 (logits of
+std ~0.06 at the 0.02-std weights).  bf16 inputs with d in {64, 128}, hidden
+in {128, 256} and 16-byte aligned rows take the tensor-core kernel (W1 split
+into two bf16 parts, fp32 accumulation); other layouts take the fp32
+CUDA-core kernels."""
 import numpy as np
 import pytest
 import torch
@@ -23,7 +26,9 @@ def _run(K, V, W1, W2):
 
 
 @pytest.mark.parametrize("N,Hkv,d,hidden", [(1000, 8, 128, 256), (333, 2, 64, 256),
-                                            (257, 3, 128, 300), (64, 1, 128, 1)])
+                                            (257, 3, 128, 300), (64, 1, 128, 1),
+                                            (1, 1, 64, 128), (129, 4, 128, 128),
+                                            (5000, 2, 64, 128)])
 def test_matches_oracle(N, Hkv, d, hidden, cuda_device):
     _, Kb, Vb = gen_qkv(N, N, Hkv, Hkv, d, 500000.0)
     rng = np.random.default_rng(hidden)
@@ -78,3 +83,38 @@ def test_general_layout_path(d, pad, cuda_device):
     lv, ls = _run(padded(Kb), padded(Vb), W1, W2)
     rv, rs = oracle.index_scores(Kb, Vb, W1, W2)
     assert np.abs(lv - rv).max() <= TOL and np.abs(ls - rs).max() <= TOL
+
+
+@pytest.mark.parametrize("d,hidden", [(128, 256), (64, 128)])
+def test_tensor_core_path_padded_rows(d, hidden, cuda_device):
+    # token stride Hkv*d + 8 bf16 (still on the 16-byte grid): the tensor-core
+    # kernel must follow the stride, not assume packed rows
+    N, Hkv, pad = 700, 3, 8
+    _, Kb, Vb = gen_qkv(d + hidden, N, Hkv, Hkv, d, 500000.0)
+    rng = np.random.default_rng(d + hidden)
+    W1 = (0.02 * rng.standard_normal((hidden, 2 * d))).astype(np.float32)
+    W2 = (0.02 * rng.standard_normal((2, hidden))).astype(np.float32)
+
+    def padded(bits):
+        buf = torch.zeros((N, Hkv * d + pad), dtype=torch.int16)
+        buf[:, : Hkv * d] = torch.from_numpy(bits.reshape(N, Hkv * d).view(np.int16))
+        return buf.cuda().view(torch.bfloat16).as_strided((N, Hkv, d), (Hkv * d + pad, d, 1))
+
+    lv, ls = _run(padded(Kb), padded(Vb), W1, W2)
+    rv, rs = oracle.index_scores(Kb, Vb, W1, W2)
+    assert np.abs(lv - rv).max() <= TOL and np.abs(ls - rs).max() <= TOL
+
+
+def test_deterministic_across_runs(cuda_device):
+    # two hidden slices add into each logit: with exactly two addends onto
+    # zero the result does not depend on their order
+    N, Hkv, d, hidden = 4096, 8, 128, 256
+    _, Kb, Vb = gen_qkv(11, N, Hkv, Hkv, d, 500000.0)
+    rng = np.random.default_rng(12)
+    W1 = (0.02 * rng.standard_normal((hidden, 2 * d))).astype(np.float32)
+    W2 = (0.02 * rng.standard_normal((2, hidden))).astype(np.float32)
+    K, V = bf16_to_dev(Kb), bf16_to_dev(Vb)
+    first = _run(K, V, W1, W2)
+    for _ in range(3):
+        again = _run(K, V, W1, W2)
+        assert np.array_equal(first[0], again[0]) and np.array_equal(first[1], again[1])
