@@ -37,7 +37,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from vs_workloads import BATCH_WORKLOADS, BLOCK_WORKLOADS, WORKLOADS  # noqa: E402
+from vs_workloads import BATCH_WORKLOADS, BLOCK_WORKLOADS, WORKLOADS, small_variant  # noqa: E402
 
 METRIC = "VS-sparse prefill ms/layer & effective TFLOP/s at 128K; speedup vs dense"
 UNIT = "TFLOP/s"
@@ -60,6 +60,9 @@ def parse():
     ap.add_argument("--agg-steps", type=int, default=2,
                     help="timed runs of the ground-truth aggregation pass (0: skip)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run a single-sequence workload at this many tokens instead of its own "
+                         "(same generators, caps scaled); for small profiling cases")
     return ap.parse_args()
 
 
@@ -403,6 +406,23 @@ def run_ours(args, w):
     job_flops = sum_over_ranks([flops], dev)[0] if sharded else world * flops
     value = job_flops / (ms_step * 1e-3) / 1e12
 
+    # the indexer alone, launches queued back to back: the in-step figure above
+    # also holds the host's marshalling before its first launch (the GPU waits
+    # for it after the L2 flush); the K/V rows it reads exceed L2
+    ms_idx_kernel = None
+    if w.indexer:
+        n_idx = 5
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        vs.vs_index_scores(K, V, W1d, W2d, LV, LS)
+        a.record(stream)
+        for _ in range(n_idx):
+            vs.vs_index_scores(K, V, W1d, W2d, LV, LS)
+        b.record(stream)
+        b.synchronize()
+        ms_idx_kernel = a.elapsed_time(b) / n_idx
+
     # dense causal kernel on the same inputs (speed-up denominator)
     ws_dense = vs.workspace(256, dev)
     dense_ms = None
@@ -597,9 +617,11 @@ def run_ours(args, w):
                    "l2": "inputs exceed L2 (Q/K/V/O resident in HBM) and a 256 MiB buffer is "
                          "written between timed steps, outside the timed windows"},
         "ms_per_layer": round(ms_step, 3), "ms_indexer": round(ms_idx, 3) if w.indexer else None,
+        "ms_indexer_back_to_back": round(ms_idx_kernel, 3) if w.indexer else None,
         "ms_select": round(ms_sel, 3), "ms_attention": round(ms_att, 3),
         "kernels": kernel_rooflines(w, peaks, N, Hq, Hkv, d, H_sel, flops, algo_bytes, ms_att,
-                                    ms_sel, ms_idx, vih.shape[1], sih.shape[1], agg),
+                                    ms_sel, ms_idx_kernel if w.indexer else ms_idx, vih.shape[1],
+                                    sih.shape[1], agg),
         "selected_pairs": int(P_total), "density_vs_causal": round(P_total / (Hq * N * (N + 1) / 2), 5),
         "dense_ms": None if dense_ms is None else round(dense_ms, 3),
         "dense_tflops": None if dense_ms is None else round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
@@ -1294,6 +1316,8 @@ def main():
             run_batch(args, BATCH_WORKLOADS[args.workload])
         return
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = small_variant(w, args.tokens)
     if args.impl == "reference":
         run_reference(args, w)
     else:

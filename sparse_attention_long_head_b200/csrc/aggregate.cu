@@ -375,26 +375,14 @@ __global__ void __launch_bounds__(kAggThreads, 1)
   }
 }
 
-void encode_map_agg(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t inner,
-                    int64_t rows, int64_t row_stride_elems, CUresult* rc) {
-  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)row_stride_elems * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) *rc = r;
-}
-
 template <int D>
 cudaError_t launch_agg_impl(const AggArgs& a) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap mQ, mK;
   CUresult rc = CUDA_SUCCESS;
-  encode_map_agg(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.N, a.q_stride, &rc);
-  encode_map_agg(enc, &mK, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, &rc);
+  encode_rows_bf16_sw128(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.N, a.q_stride, &rc);
+  encode_rows_bf16_sw128(enc, &mK, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, &rc);
   if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
   AggParams P;
   P.N = a.N;

@@ -13,14 +13,16 @@
 // heads contiguous in a token row, 16-byte aligned rows) runs X W1^T on the
 // tensor cores: W1 = hi + lo with hi = bf16(W1) and lo = bf16(W1 - hi)
 // (residual below 2^-17 of |W1|), and X W1^T = X hi^T + X lo^T as two bf16
-// MMAs with fp32 accumulation (bf16 x bf16 products are exact in fp32).  Persistent CTAs
-// each keep one 128-unit hidden slice of both parts in shared memory (128-
-// byte-swizzled, K-major), stage a 128-token X tile per step with 16-byte
-// loads, and accumulate the 128 x 128 tile in TMEM; the epilogue applies ReLU
-// and the slice's share of the down-projection and adds it to the logits
-// (zeroed first; at most two slices, so the order of the two additions does
-// not change the sum).  A device wait that runs out (a correct launch never
-// does) leaves NaN in the logits of that tile and of the CTA's later tiles.
+// MMAs with fp32 accumulation (bf16 x bf16 products are exact in fp32).
+// Persistent CTAs each keep one 128-unit hidden slice of both parts in shared
+// memory (128-byte-swizzled, K-major).  TMA streams the 128-token X tiles
+// through a ring of 64-feature boxes; the MMAs accumulate each 128 x 128 tile
+// in one of two TMEM accumulators, so that the epilogue of one tile overlaps
+// the MMAs of the next.  The epilogue applies ReLU and the slice's share of
+// the down-projection and adds it to the logits (zeroed first; at most two
+// slices, so the order of the two additions does not change the sum).  A
+// device wait that runs out (a correct launch never does) leaves NaN in the
+// logits of that tile and of the CTA's later tiles.
 //
 // index_scores_vec_kernel is the same computation for aligned inputs (16-byte
 // aligned rows, d a multiple of 16): a CTA takes 128 consecutive tokens of
@@ -274,24 +276,42 @@ __global__ void __launch_bounds__(kIdxThreads) index_scores_vec_kernel(IdxArgs a
   }
 }
 
-constexpr int kTcThreads = 128;
+// Roles of the tensor-core kernel: warp 0 issues the TMA loads, warp 1 owns
+// TMEM and issues the MMAs, warps 2..5 run the epilogue (warp w reads TMEM
+// lanes 32 (w mod 4) .. 32 (w mod 4) + 31, as the hardware requires).
+constexpr int kTcWarps = 6;
+constexpr int kTcThreads = 32 * kTcWarps;
+constexpr int kTcEpiThreads = 128;
 constexpr uint64_t kTcWaitNs = kDefaultWaitLimitNs;
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1) index_scores_tc_kernel(IdxArgs a, int slices) {
-  constexpr int KB = 2 * D / 64;       // 64-feature boxes of one [k; v] row
-  constexpr int kBox = 128 * 128;      // bytes of a 128-row x 64-bf16 box
+struct IdxTc {
+  static constexpr int KB = 2 * D / 64;                // 64-feature boxes of one [k; v] row
+  static constexpr int kBox = 128 * 128;               // bytes of a 128-row x 64-bf16 box
+  static constexpr int kStages = D == 128 ? 5 : 8;     // X ring, one box per stage
+  static constexpr int kSmem = (2 * KB + kStages) * kBox + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, IdxArgs a, int slices) {
+  using C = IdxTc<D>;
+  constexpr int KB = C::KB, kBox = C::kBox, S = C::kStages;
   extern __shared__ uint8_t dyn_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sW = smem;                  // [2 parts][KB boxes]
-  uint8_t* sX = smem + 2 * KB * kBox;  // [KB boxes]
+  uint8_t* sW = smem;                  // [2 parts][KB boxes] of the W1 slice
+  uint8_t* sR = smem + 2 * KB * kBox;  // X ring: S boxes
   __shared__ float w2s[2][128];
-  __shared__ __align__(8) uint64_t mma_bar;
+  // full[S], empty[S], accfull[2], accempty[2], drain
+  __shared__ __align__(8) uint64_t bars[2 * S + 5];
   __shared__ uint32_t tslot;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  __shared__ int abort_flag, status_sink;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.x % slices;   // hidden slice [128 j, 128 j + 128)
   const int D2 = 2 * D;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
   // W1 slice -> hi / lo bf16 parts, 8 features (one 16-byte chunk) at a time
   for (int e = tid; e < 128 * (D2 / 8); e += kTcThreads) {
     const int n = e / (D2 / 8), c = (e % (D2 / 8)) * 8;
@@ -311,68 +331,112 @@ __global__ void __launch_bounds__(kTcThreads, 1) index_scores_tc_kernel(IdxArgs 
     *reinterpret_cast<uint4*>(sW + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(sW + KB * kBox + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
-  for (int e = tid; e < 256; e += kTcThreads) w2s[e / 128][e % 128] = a.W2[(e / 128) * a.hidden + 128 * j + e % 128];
+  for (int e = tid; e < 256; e += kTcThreads)
+    w2s[e / 128][e % 128] = a.W2[(e / 128) * a.hidden + 128 * j + e % 128];
   if (tid == 0) {
-    mbar_init(smem_u32(&mma_bar), 1);
+    for (int i = 0; i < 2 * S; ++i) mbar_init(bar(i), 1);
+    mbar_init(bar(2 * S), 1);
+    mbar_init(bar(2 * S + 1), 1);
+    mbar_init(bar(2 * S + 2), kTcEpiThreads);
+    mbar_init(bar(2 * S + 3), kTcEpiThreads);
+    mbar_init(bar(2 * S + 4), 1);
+    abort_flag = 0;
+    status_sink = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(&tslot), 128);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tslot), 256);  // two 128-column accumulators
     tmem_relinquish();
   }
-  fence_proxy_async_smem();
+  fence_proxy_async_smem();  // the W1 parts, written by threads, are read by the tensor core
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tacc = tslot;
-  constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
-  const uint64_t xdesc = sdesc_sw128(smem_u32(sX), 16, 1024);
-  const uint64_t wdesc = sdesc_sw128(smem_u32(sW), 16, 1024);
-  const int64_t ntile = (a.N + 127) / 128;
-  const int64_t items = ntile * a.Hkv;
-  const int per = gridDim.x / slices;  // CTAs per slice
-  uint32_t phase = 0;
-  bool dead = false;  // CTA-uniform: a wait for this CTA's MMAs ran out
-  for (int64_t it = blockIdx.x / slices; it < items; it += per) {
-    const int g = (int)(it % a.Hkv);
-    const int64_t t0 = (it / a.Hkv) * 128;
-    float pv = __int_as_float(0x7fc00000), ps = pv;  // NaN unless the tile completes
-    if (!dead) {
-      // X tile: 128 tokens x [k; v], 16-byte chunks into the swizzled boxes
-      for (int e = tid; e < 128 * (D2 / 8); e += kTcThreads) {
-        const int r = e / (D2 / 8), c = (e % (D2 / 8)) * 8;
-        const int64_t t = t0 + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (t < a.N) {
-          const uint16_t* base = static_cast<const uint16_t*>(c < D ? a.K : a.V);
-          v = __ldg(reinterpret_cast<const uint4*>(base + t * a.stride_tok + (int64_t)g * D + (c % D)));
-        }
-        *reinterpret_cast<uint4*>(sX + (c / 64) * kBox + sw128_off(r, (c % 64) / 8)) = v;
-      }
-      fence_proxy_async_smem();  // generic-proxy stores -> the tensor core's reads
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int p = 0; p < 2; ++p)
-#pragma unroll
-          for (int kk = 0; kk < D2 / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
-            mma_ss(tacc, xdesc + off, wdesc + ((p * KB * kBox) >> 4) + off, idesc,
-                   (p | kk) ? 1u : 0u);
+  const uint32_t tbase = tslot;
+  // the index launch has no status word: a timeout shows as NaN logits
+  const WaitCtx wc{kTcWaitNs, &status_sink, &abort_flag};
+  const int64_t items = (int64_t)((a.N + 127) / 128) * a.Hkv;  // (token tile, KV head)
+  const int per = gridDim.x / slices;
+  const int64_t first = blockIdx.x / slices;
+  const int nmine = first < items ? (int)((items - 1 - first) / per + 1) : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int q = 0;  // boxes issued
+      bool live = true;
+      for (int i = 0; i < nmine && live; ++i) {
+        const int64_t it = first + (int64_t)i * per;
+        const int g = (int)(it % a.Hkv);
+        const int y = (int)((it / a.Hkv) * 128);
+        for (int b = 0; b < KB; ++b) {
+          const int st = q % S;
+          if (q >= S && !mbar_wait(bar(S + st), (q / S - 1) & 1, wc)) {
+            live = false;
+            break;
           }
-        mma_commit(smem_u32(&mma_bar));
+          mbar_arrive_expect_tx(bar(st), kBox);
+          tma_load_2d(smem_u32(sR + st * kBox), b < KB / 2 ? &tmK : &tmV, bar(st),
+                      g * D + (b % (KB / 2)) * 64, y);
+          ++q;
+        }
       }
+      // copies still in flight land before the CTA exits (at once unless aborted)
+      for (int r = q > S ? q - S : 0; r < q; ++r) mbar_wait_drain(bar(r % S), (r / S) & 1, kTcWaitNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+      const uint64_t wdesc = sdesc_sw128(smem_u32(sW), 16, 1024);
+      int q = 0;  // boxes consumed
+      bool live = true;
+      for (int i = 0; i < nmine && live; ++i) {
+        const int acc = i & 1;
+        if (i >= 2 && !mbar_wait(bar(2 * S + 2 + acc), ((i >> 1) - 1) & 1, wc)) break;
+        tc_fence_after();
+        const uint32_t tacc = tbase + acc * 128;
+        for (int b = 0; b < KB; ++b, ++q) {
+          const int st = q % S;
+          if (!mbar_wait(bar(st), (q / S) & 1, wc)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t xdesc = sdesc_sw128(smem_u32(sR + st * kBox), 16, 1024);
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tacc, xdesc + ((kk * 32) >> 4), wdesc + (((p * KB + b) * kBox + kk * 32) >> 4),
+                     idesc, (b | p | kk) ? 1u : 0u);
+          mma_commit(bar(S + st));  // the box's slot is free once these MMAs have read it
+        }
+        if (live) mma_commit(bar(2 * S + acc));
+      }
+      // every MMA issued has finished before TMEM is released
+      mma_commit(bar(2 * S + 4));
+      mbar_wait_drain(bar(2 * S + 4), 0, kTcWaitNs);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    bool live = true;
+    for (int i = 0; i < nmine; ++i) {
+      const int64_t it = first + (int64_t)i * per;
+      const int g = (int)(it % a.Hkv);
+      const int64_t t = (it / a.Hkv) * 128 + row;
+      const int acc = i & 1;
+      float pv = __int_as_float(0x7fc00000), ps = pv;  // NaN unless the tile completes
       // warp-uniform, since tcgen05.ld is a warp-wide instruction
-      const bool ok = __all_sync(0xffffffffu, mbar_wait_drain(smem_u32(&mma_bar), phase, kTcWaitNs));
-      tc_fence_after();
-      if (ok) {
-        // epilogue: thread tid = token row; TMEM lanes 32 warp .. 32 warp + 31
+      if (live) live = __all_sync(0xffffffffu, mbar_wait(bar(2 * S + acc), (i >> 1) & 1, wc));
+      if (live) {
+        tc_fence_after();
         pv = ps = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t v[32];
-          tmem_ld32(tacc + ((uint32_t)(warp * 32) << 16) + 32 * q, v);
+          tmem_ld32(tbase + acc * 128 + ((uint32_t)(quarter * 32) << 16) + 32 * q, v);
           tmem_ld_wait(v);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -381,23 +445,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) index_scores_tc_kernel(IdxArgs 
             ps = fmaf(w2s[1][32 * q + c], h, ps);
           }
         }
+        tc_fence_before();
+        mbar_arrive(bar(2 * S + 2 + acc));
       }
-      tc_fence_before();
-      // TMEM and the X tile are reused by the next tile
-      dead = __syncthreads_or(!ok) != 0;
-      if (!dead) phase ^= 1u;
-    }
-    const int64_t t = t0 + tid;
-    if (t < a.N) {
-      atomicAdd(&a.lv[(int64_t)g * a.N + t], pv);
-      atomicAdd(&a.ls[(int64_t)g * a.N + t], ps);
+      if (t < a.N) {
+        atomicAdd(&a.lv[(int64_t)g * a.N + t], pv);
+        atomicAdd(&a.ls[(int64_t)g * a.N + t], ps);
+      }
     }
   }
-  // after a timeout, let the MMAs in flight land before TMEM is released
-  if (dead) mbar_wait_drain(smem_u32(&mma_bar), phase, kTcWaitNs);
-  if (warp == 0) {
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tacc, 128);
+    tmem_dealloc(tbase, 256);
   }
 }
 
@@ -412,9 +473,14 @@ cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, 
                   stride_head == d && (stride_tok * 2) % 16 == 0 && al16(K) && al16(V) &&
                   al16(W1);
   if (tc) {
+    EncodeTiledFn enc = get_encode_tiled();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap mK, mV;
+    CUresult rc = CUDA_SUCCESS;
+    encode_rows_bf16_sw128(enc, &mK, K, (int64_t)Hkv * d, N, stride_tok, &rc);
+    encode_rows_bf16_sw128(enc, &mV, V, (int64_t)Hkv * d, N, stride_tok, &rc);
+    if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int slices = hidden / 128;
-    const int kb = 2 * d / 64;
-    const size_t smem = (size_t)3 * kb * 128 * 128 + 1024;  // W1 hi / lo parts, X tile, alignment
     if (cudaMemsetAsync(lv, 0, sizeof(float) * (size_t)N * Hkv, stream) != cudaSuccess ||
         cudaMemsetAsync(ls, 0, sizeof(float) * (size_t)N * Hkv, stream) != cudaSuccess)
       return cudaErrorUnknown;
@@ -425,14 +491,14 @@ cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, 
     cudaError_t e;
     if (d == 128) {
       e = cudaFuncSetAttribute(index_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+                               IdxTc<128>::kSmem);
       if (e != cudaSuccess) return e;
-      index_scores_tc_kernel<128><<<grid, kTcThreads, smem, stream>>>(a, slices);
+      index_scores_tc_kernel<128><<<grid, kTcThreads, IdxTc<128>::kSmem, stream>>>(mK, mV, a, slices);
     } else {
       e = cudaFuncSetAttribute(index_scores_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+                               IdxTc<64>::kSmem);
       if (e != cudaSuccess) return e;
-      index_scores_tc_kernel<64><<<grid, kTcThreads, smem, stream>>>(a, slices);
+      index_scores_tc_kernel<64><<<grid, kTcThreads, IdxTc<64>::kSmem, stream>>>(mK, mV, a, slices);
     }
     return cudaGetLastError();
   }

@@ -241,5 +241,10 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn get_encode_tiled();
 int device_sm_count();
+// 2-D bf16 map over `rows` rows of `inner` elements (row stride in elements),
+// box of 128 rows x 64 elements, 128-byte swizzle, zero fill past the edges.
+// Leaves *rc unchanged on success.
+void encode_rows_bf16_sw128(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t inner,
+                            int64_t rows, int64_t row_stride_elems, CUresult* rc);
 
 }  // namespace vs
