@@ -17,6 +17,13 @@
 //     of counts and, for the threshold rule, of fp64 softmax mass; the cluster
 //     merges them through distributed shared memory, and every CTA takes the
 //     same decision from the same merged data.
+//   * The mass histogram takes no fp64 atomics (which the hardware runs as
+//     compare-and-swap loops): each warp owns a private copy; lanes holding
+//     the same digit are grouped with a match instruction and summed in a
+//     tree over their ranks, and each group's lowest lane adds the sum with
+//     a plain read-modify-write (distinct groups touch distinct buckets).
+//     The CTA's histogram is the warps' copies added in warp order, so the
+//     whole sum is in a fixed order and the selection is deterministic.
 //   * The threshold rule walks the buckets from the top, accumulating mass
 //     until tau * Z is reached (Z = the total of the first pass's mass
 //     histogram); inside the final group of equal keys the count follows from
@@ -120,6 +127,25 @@ __device__ __forceinline__ int block_excl_scan(int v, int* buf) {
   return r;
 }
 
+// Sum of v over the lanes in `peers` (this lane's group, from
+// __match_any_sync; every lane of the warp calls this).  A binary tree over
+// the group's ranks: at step s the lane of rank r (r a multiple of 2s) adds
+// the partial sum of rank r + s.  The group's total ends in its lowest lane
+// (rank 0).  `steps` = ceil(log2(largest group in the warp)), warp-uniform.
+__device__ __forceinline__ double group_sum(unsigned peers, double v, int steps) {
+  const int lane = threadIdx.x & 31;
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  const unsigned above = lane == 31 ? 0u : peers & ~((2u << lane) - 1u);  // peers after me
+  for (int i = 0, st = 1; i < steps; ++i, st <<= 1) {
+    unsigned r = above;  // the peer of rank rank + st: the st-th set bit of `above`
+    for (int j = 1; j < st && r; ++j) r &= r - 1u;
+    const unsigned src = r ? (unsigned)(__ffs(r) - 1) : 32u;
+    const double t = __shfl_sync(0xffffffffu, v, src < 32u ? src : (unsigned)lane);
+    if ((rank & (2 * st - 1)) == 0 && src < 32u) v += t;
+  }
+  return v;
+}
+
 template <bool CACHE>
 __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   cg::cluster_group cl = cg::this_cluster();
@@ -129,6 +155,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   const int tid = threadIdx.x, nt = blockDim.x;
   extern __shared__ uint32_t skeys[];
   __shared__ SelShared sh;
+  // per-warp mass histograms [warp][256], after the key cache (threshold rule only)
+  double* wmass = reinterpret_cast<double*>(skeys + (CACHE ? (a.chunk + 1) / 2 * 2 : 0));
 
   const float* row = a.scores + (int64_t)h * a.ld;
   const int lo = rank * a.chunk;
@@ -222,15 +250,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
     if (tid < 256) {
       sh.cnt_c[buf][tid] = 0;
       sh.cnt_t[buf][tid] = 0;
-      sh.mass_t[buf][tid] = 0.0;
     }
+    if (use_mass)
+      for (int i = tid; i < (kSelThreads / 32) * 256; i += nt) wmass[i] = 0.0;
     __syncthreads();
-    // Run-length aggregation per search: keys of a pass often fall in one
+    // Count path: run-length aggregation (keys of a pass often fall in one
     // bucket, so a thread accumulates while its bucket repeats and flushes on
-    // change; the final flush is reduced across the warp when all lanes agree.
-    int cur_c = -1, cur_t = -1;
-    uint32_t rc_c = 0, rc_t = 0;
-    double rm_t = 0.0;
+    // change; the final flush is reduced across the warp when all lanes agree).
+    int cur_c = -1;
+    uint32_t rc_c = 0;
     for (int e = tid; e < n; e += nt) {
       const uint32_t k = key_at(e);
       if ((k & pm_c) == pf_c) {
@@ -241,20 +269,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
           rc_c = 0;
         }
         ++rc_c;
-      }
-      if (use_mass && (k & pm_t) == pf_t) {
-        const int dg = (k >> shift) & 255;
-        if (dg != cur_t) {
-          if (cur_t >= 0) {
-            atomicAdd(&sh.cnt_t[buf][cur_t], rc_t);
-            atomicAdd(&sh.mass_t[buf][cur_t], rm_t);
-          }
-          cur_t = dg;
-          rc_t = 0;
-          rm_t = 0.0;
-        }
-        ++rc_t;
-        rm_t += pmass(k, kmax, smax);
       }
     }
     __syncwarp();
@@ -267,18 +281,50 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
         atomicAdd(&sh.cnt_c[buf][cur_c], rc_c);
       }
     }
+    // Mass path: a warp takes 32 consecutive keys per step (warp-uniform trip
+    // count); lanes with equal digits form a group, whose lowest lane adds the
+    // group's count (shared atomic, integer) and mass (the warp's own
+    // histogram, plain add: the groups' digits differ).
     if (use_mass) {
-      const int c0 = __shfl_sync(0xffffffffu, cur_t, 0);
-      if (__all_sync(0xffffffffu, cur_t == c0) && c0 >= 0) {
-        const uint32_t r = __reduce_add_sync(0xffffffffu, rc_t);
-        for (int o = 16; o > 0; o >>= 1) rm_t += __shfl_xor_sync(0xffffffffu, rm_t, o);
-        if ((tid & 31) == 0) {
-          atomicAdd(&sh.cnt_t[buf][c0], r);
-          atomicAdd(&sh.mass_t[buf][c0], rm_t);
+      const int lane = tid & 31;
+      double* wm = wmass + (tid >> 5) * 256;
+      for (int base = tid - lane; base < n; base += nt) {
+        const int e = base + lane;
+        int dg = 256;  // 256: not in the searched prefix (or past the end)
+        double m = 0.0;
+        if (e < n) {
+          const uint32_t k = key_at(e);
+          if ((k & pm_t) == pf_t) {
+            dg = (k >> shift) & 255;
+            m = pmass(k, kmax, smax);
+          }
         }
-      } else if (cur_t >= 0) {
-        atomicAdd(&sh.cnt_t[buf][cur_t], rc_t);
-        atomicAdd(&sh.mass_t[buf][cur_t], rm_t);
+        if (__all_sync(0xffffffffu, dg == __shfl_sync(0xffffffffu, dg, 0))) {
+          // one digit across the warp (the usual case in the first pass)
+          if (dg < 256) {
+            for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
+            if (lane == 0) {
+              atomicAdd(&sh.cnt_t[buf][dg], 32u);
+              wm[dg] += m;
+            }
+          }
+          continue;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, dg);
+        const int gsize = __popc(peers);
+        const int gmax = __reduce_max_sync(0xffffffffu, (unsigned)gsize);
+        const int steps = 32 - __clz(gmax - 1);  // ceil(log2(gmax)); 0 for gmax = 1
+        m = group_sum(peers, m, steps);
+        if (dg < 256 && (peers & ((1u << lane) - 1u)) == 0) {
+          atomicAdd(&sh.cnt_t[buf][dg], (uint32_t)gsize);
+          wm[dg] += m;
+        }
+      }
+      __syncthreads();
+      if (tid < 256) {  // the CTA's histogram: the warps' copies in warp order
+        double t = 0.0;
+        for (int w = 0; w < kSelThreads / 32; ++w) t += wmass[w * 256 + tid];
+        sh.mass_t[buf][tid] = t;
       }
     }
     cl.sync();
@@ -425,6 +471,16 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
                           cudaStream_t stream) {
   int C = (N + 4095) / 4096;
   C = C < 1 ? 1 : (C > kSelMaxCluster ? kSelMaxCluster : C);
+  {
+    // Many heads: a cluster per head at this size needs more than one wave of
+    // SMs (one CTA per SM).  The smallest cluster whose CTAs still cache their
+    // slice of the keys may fit all heads in one wave; take it then.
+    int cmin = (N + kSelCacheKeys - 1) / kSelCacheKeys;
+    cmin = cmin < 1 ? 1 : cmin;
+    const int sms = device_sm_count();
+    if (cmin < C && H * C > sms && H * cmin <= sms) C = cmin;
+  }
+  const size_t mass_bytes = mode == VS_SELECT_THRESHOLD ? sizeof(double) * (kSelThreads / 32) * 256 : 0;
   // Few heads leave most SMs idle: split long rows over 16-CTA clusters (a
   // non-portable size: used only when the device can place such a cluster).
   bool wide = C == kSelMaxCluster && H * kSelMaxCluster * 2 <= device_sm_count() &&
@@ -436,7 +492,7 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
     cudaLaunchConfig_t probe = {};
     probe.gridDim = dim3(16, H, 1);
     probe.blockDim = dim3(kSelThreads, 1, 1);
-    probe.dynamicSmemBytes = cache16 ? sizeof(uint32_t) * chunk16 : 0;
+    probe.dynamicSmemBytes = (cache16 ? sizeof(uint32_t) * ((chunk16 + 1) / 2 * 2) : 0) + mass_bytes;
     cudaLaunchAttribute pa[1];
     pa[0].id = cudaLaunchAttributeClusterDimension;
     pa[0].val.clusterDim.x = 16;
@@ -462,7 +518,7 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, H, 1);
   cfg.blockDim = dim3(kSelThreads, 1, 1);
-  cfg.dynamicSmemBytes = cache ? sizeof(uint32_t) * chunk : 0;
+  cfg.dynamicSmemBytes = (cache ? sizeof(uint32_t) * ((chunk + 1) / 2 * 2) : 0) + mass_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -483,6 +539,9 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
     }
     e = cudaLaunchKernelEx(&cfg, select_kernel<true>, a);
   } else {
+    e = cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)cfg.dynamicSmemBytes);
+    if (e != cudaSuccess) return e;
     if (wide) {
       e = cudaFuncSetAttribute(select_kernel<false>,
                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
