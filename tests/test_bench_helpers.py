@@ -93,3 +93,32 @@ def test_indexer_roofline_terms():
     assert k["indexer"]["bound"] == ("tensor" if flops / 1.5e15 >= nbytes / 6e12 else "hbm")
     assert abs(k["indexer"]["frac"] - round(t / 2e-3, 4)) < 1e-12
     assert abs(k["indexer"]["achieved_gbs"] - round(nbytes / 2e-3 / 1e9, 1)) < 1e-9
+
+
+def test_e2e_unit_order():
+    # two heavy and two light KV groups of 2 heads; copies cost about as much as a
+    # light group's compute.  The chosen order covers every head once, splits the
+    # first and last group into heads, and is no longer (in the model) than
+    # heaviest-first, which leaves the light groups' copies out for the end.
+    Hkv, G = 4, 2
+    head_cost = [8.0, 8.0, 0.2, 0.2, 8.0, 8.0, 0.2, 0.2]
+    units = bench.e2e_units(Hkv, G, head_cost, 1.0, 2.0, 1.0)
+    heads = sorted(h for _, h0, h1 in units for h in range(h0, h1))
+    assert heads == list(range(Hkv * G))
+    assert units[0][2] - units[0][1] == 1 and units[-1][2] - units[-1][1] == 1
+    first, last = units[0][0], units[-1][0]
+    assert head_cost[first * G] == 8.0 and head_cost[last * G] == 8.0
+
+    def model(us):
+        t_in = t_c = t_out = 0.0
+        seen = set()
+        for g, h0, h1 in us:
+            t_in += (h1 - h0) + (0.0 if g in seen else 2.0)
+            seen.add(g)
+            t_c = max(t_c, t_in) + sum(head_cost[h0:h1]) + 0.05
+            t_out = max(t_out, t_c) + (h1 - h0)
+        return t_out
+
+    hf_units = [(0, 0, 1), (0, 1, 2), (2, 4, 6), (1, 2, 4), (3, 6, 7), (3, 7, 8)]
+    assert model(units) <= model(hf_units)
+    assert model(units) < model(hf_units) - 0.5
