@@ -177,8 +177,16 @@ __global__ void __launch_bounds__(kAggThreads, 1)
       }
       int64_t carry_off = -1;
       float carry = 0.f;
+      // this row's LSE for the walk's next tile, loaded a tile ahead
+      auto lse_of = [&](int s) -> float {
+        const int64_t ii = 128 * (int64_t)(a.b + agg_tile(a, grp, s)) + r;
+        return ii < P.N ? __ldg(lse_h + ii) : 0.f;
+      };
+      float lse_next = ng > 0 ? lse_of(0) : 0.f;
       for (int s = 0; s < ng && ok; ++s, ++cnt) {
         const int j = agg_tile(a, grp, s);
+        const float lse_i = lse_next;
+        if (s + 1 < ng) lse_next = lse_of(s + 1);
         bool w = mbar_wait(bar(B_SFULL + grp), cnt & 1, wc);
         __syncwarp();
         if (!named_bar_and(gbar, 128, w)) {
@@ -197,7 +205,7 @@ __global__ void __launch_bounds__(kAggThreads, 1)
         mbar_arrive(bar(B_SEMPTY + grp));  // the S buffer may be overwritten
         const int64_t i = 128 * (int64_t)(a.b + j) + r;
         // rows past N weigh nothing (their Q rows are zero-filled, so s is finite)
-        const float nl = i < P.N ? -__ldg(lse_h + i) * 1.4426950408889634f : -INFINITY;
+        const float nl = i < P.N ? -lse_i * 1.4426950408889634f : -INFINITY;
         if (j == 0) {  // the diagonal tile: keys after the row weigh nothing
 #pragma unroll
           for (int q = 0; q < 4; ++q)
