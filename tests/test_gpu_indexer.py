@@ -118,3 +118,29 @@ def test_deterministic_across_runs(cuda_device):
     for _ in range(3):
         again = _run(K, V, W1, W2)
         assert np.array_equal(first[0], again[0]) and np.array_equal(first[1], again[1])
+
+
+@pytest.mark.parametrize("d,hidden", [(128, 256), (64, 128)])
+def test_tensor_core_single_weight_probes(d, hidden, cuda_device):
+    # one nonzero bf16-representable weight: the split has no low part, the
+    # MMA sums a single exact product, so the logits are exact -- any slip in
+    # the swizzled operand layout or the hidden-slice split moves the weight
+    # to another feature or unit
+    N, Hkv = 300, 2
+    _, Kb, Vb = gen_qkv(5, N, Hkv, Hkv, d, 500000.0)
+    k = (Kb.astype(np.uint32) << 16).view(np.float32)
+    v = (Vb.astype(np.uint32) << 16).view(np.float32)
+    K, V = bf16_to_dev(Kb), bf16_to_dev(Vb)
+    for (u, c, r, w1, w2) in [(0, 0, 0, 1.0, 1.0), (hidden - 1, 2 * d - 1, 1, -2.0, 0.5),
+                              (hidden // 2 + 3, d, 0, 1.5, -1.0), (77 % hidden, d - 1, 1, 1.0, 3.0),
+                              (hidden // 2 - 1, 37, 0, 0.25, 2.0)]:
+        W1 = np.zeros((hidden, 2 * d), np.float32)
+        W2 = np.zeros((2, hidden), np.float32)
+        W1[u, c] = w1
+        W2[r, u] = w2
+        lv, ls = _run(K, V, W1, W2)
+        x = k[..., c] if c < d else v[..., c - d]  # [N, Hkv]
+        want = (np.float32(w2) * np.maximum(np.float32(w1) * x, np.float32(0))).T.astype(np.float64)
+        got, other = (lv, ls) if r == 0 else (ls, lv)
+        np.testing.assert_array_equal(got, want)
+        assert np.all(other == 0.0)
