@@ -241,7 +241,10 @@ class ClockSampler:
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # raw samples: $VS_CLOCK_DIR if set (to keep them), else the temp directory
+        import tempfile
+        d = os.environ.get("VS_CLOCK_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"vs_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
