@@ -481,14 +481,14 @@ cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, 
     encode_rows_bf16_sw128(enc, &mV, V, (int64_t)Hkv * d, N, stride_tok, &rc);
     if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int slices = hidden / 128;
-    if (cudaMemsetAsync(lv, 0, sizeof(float) * (size_t)N * Hkv, stream) != cudaSuccess ||
-        cudaMemsetAsync(ls, 0, sizeof(float) * (size_t)N * Hkv, stream) != cudaSuccess)
-      return cudaErrorUnknown;
+    cudaError_t e = cudaMemsetAsync(lv, 0, sizeof(float) * (size_t)N * Hkv, stream);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(ls, 0, sizeof(float) * (size_t)N * Hkv, stream);
+    if (e != cudaSuccess) return e;
     const int64_t items = ((int64_t)N + 127) / 128 * Hkv;
     int grid = device_sm_count() / slices * slices;
     if ((int64_t)grid > items * slices) grid = (int)(items * slices);
     if (grid < slices) grid = slices;
-    cudaError_t e;
     if (d == 128) {
       e = cudaFuncSetAttribute(index_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                IdxTc<128>::kSmem);
