@@ -88,8 +88,15 @@ int vs_version(void);
  *             `stride_tok`, head stride `stride_head` (elements).
  *   W1        fp32 [hidden][2d] row-major (device).   W2  fp32 [2][hidden].
  *   hidden    1..1024.
- *   logits_v, logits_s   fp32 [Hkv][N] outputs (device).
- * Computes in fp32 with fp32 accumulation.
+ *   logits_v, logits_s   fp32 [Hkv][N] outputs (device), fully overwritten.
+ * Arithmetic: bf16 K/V with d = 64 or 128, hidden = 128 or 256, stride_head
+ * = d and 16-byte aligned rows run on the tensor cores.  There W1 is split
+ * into two bf16 parts (hi = bf16(W1), lo = bf16(W1 - hi)), the products are
+ * exact and the accumulation is fp32; the result is deterministic (at most
+ * two partial sums per logit, added onto zero).  Other inputs run in fp32 on
+ * the CUDA cores.  The tensor-core kernel's device waits are bounded; a wait
+ * that runs out (never on a correct launch) leaves NaN in the logits of the
+ * tiles it affects, since this call has no workspace status word.
  */
 vs_status vs_index_scores(const void* K, const void* V, vs_dtype dtype, int N, int Hkv, int d,
                           int64_t stride_tok, int64_t stride_head, const float* W1,
