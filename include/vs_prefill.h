@@ -132,6 +132,10 @@ vs_status vs_index_scores(const void* K, const void* V, vs_dtype dtype, int N, i
  *            bytes, 256-byte aligned (holds the device status word).
  * Requires 1 <= k_or_cap <= N <= 2^20; tau in (0, 1] for THRESHOLD and
  * MAXFRAC (else VS_ERR_INVALID_ARG).
+ * The fp64 mass sums are added in a fixed order (no atomics), so repeated
+ * calls on the same scores give the same result bit for bit; where the
+ * decision lies within rounding of tau * sum_r p_r, it may differ from one
+ * taken with another summation order.
  */
 size_t vs_select_workspace_size(int H, int N);
 vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_select_mode mode,
