@@ -131,3 +131,25 @@ def test_maximum_row_length(cuda_device):
     check_select(s, TOPK, 1000)
     check_select(s, THR, N, 0.5)
     check_select(s, MAXF, 5000, 0.02)
+
+
+@pytest.mark.parametrize("H,N", [(32, 131072), (8, 262144), (3, 5000)])
+def test_threshold_repeatable_bit_for_bit(H, N, cuda_device):
+    # the fp64 mass sums have a fixed order (per-warp histograms, warp-order
+    # and rank-order merges): repeated calls give identical selections, on
+    # one-wave and two-wave cluster shapes alike
+    import torch
+    rng = np.random.default_rng(N + H)
+    s = torch.from_numpy((rng.standard_normal((H, N)) * 3.0).astype(np.float32)).cuda()
+    k = N  # no cap: the mass sums alone decide
+    ws = vs.workspace(vs.vs_select_workspace_size(H, N))
+    outs = []
+    for _ in range(3):
+        idx = torch.empty((H, k), dtype=torch.int32, device="cuda")
+        cnt = torch.empty(H, dtype=torch.int32, device="cuda")
+        vs.vs_select(s, vs.VS_SELECT_THRESHOLD, k, 0.9, idx, cnt, ws)
+        outs.append((idx.cpu().numpy(), cnt.cpu().numpy()))
+    rc, flags = vs.vs_read_device_status(ws)
+    assert rc == vs.VS_OK and flags == 0
+    for o in outs[1:]:
+        assert np.array_equal(o[0], outs[0][0]) and np.array_equal(o[1], outs[0][1])
