@@ -133,9 +133,12 @@ vs_status vs_index_scores(const void* K, const void* V, vs_dtype dtype, int N, i
  * Requires 1 <= k_or_cap <= N <= 2^20; tau in (0, 1] for THRESHOLD and
  * MAXFRAC (else VS_ERR_INVALID_ARG).
  * The fp64 mass sums are added in a fixed order (no atomics), so repeated
- * calls on the same scores give the same result bit for bit; where the
- * decision lies within rounding of tau * sum_r p_r, it may differ from one
- * taken with another summation order.
+ * calls with the same H and N on the same device give the same result bit
+ * for bit.  That order follows the thread-block cluster the launcher picks,
+ * which depends on H, N and the device's SM count: a row selected in a call
+ * with another H or N, or on another device, may be summed in another order,
+ * and where the decision lies within rounding of tau * sum_r p_r it may then
+ * differ by one entry.
  */
 size_t vs_select_workspace_size(int H, int N);
 vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_select_mode mode,
@@ -277,7 +280,10 @@ vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, 
  *   (vs_attn_workspace_size(N, Hq, H_sel, d) > 16 MiB) return
  *   VS_ERR_UNSUPPORTED before launching anything.
  *   The first call on a device resolves the array's device address with
- *   cudaGetSymbolAddress (with that device current); make that first call
+ *   cudaGetSymbolAddress (with that device current), and so does the first
+ *   call after the device's context has been replaced (cudaDeviceReset): the
+ *   address is kept per device together with the ID of the context it was
+ *   taken in.  Make the first call on a device (and the first after a reset)
  *   before any stream capture.  No cudaMalloc / cudaFree or other allocating
  *   routine is called.
  *   Every call shares the array, which keeps the last call's contents (the

@@ -7,7 +7,7 @@
 // calling cudaMalloc (which may also synchronise the device in the middle of
 // a latency-critical prefill).  This entry point serves them with a fixed
 // scratch array that every GPU loading the library holds until exit.
-#include <atomic>
+#include <mutex>
 
 #include "internal.h"
 
@@ -21,22 +21,61 @@ constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_vs_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
-static std::atomic<void*> g_scratch_addr[kMaxDevices];
 
-// Resolves (once per device, with that device current) the device address of
-// the scratch array.
+// Driver calls that identify the current context (resolved through the
+// runtime, so there is no link-time dependency on libcuda).  A context ID is
+// unique for the life of the process, so a context created after
+// cudaDeviceReset never matches the one an address was taken in.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+static void* driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
+}
+
+struct ScratchSlot {
+  unsigned long long ctx_id = 0;  // 0: not resolved yet
+  void* addr = nullptr;
+};
+static ScratchSlot g_scratch_slot[kMaxDevices];
+static std::mutex g_scratch_mu;
+
+// Resolves the device address of the scratch array for the current device,
+// once per (device, context): with that device current, on the first call
+// and again whenever the device's context has been replaced.
 static cudaError_t scratch_address(void** out) {
+  static const auto get_current = reinterpret_cast<CtxGetCurrentFn>(driver_fn("cuCtxGetCurrent"));
+  static const auto get_id = reinterpret_cast<CtxGetIdFn>(driver_fn("cuCtxGetId"));
+  if (!get_current || !get_id) return cudaErrorNotSupported;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  if (ctx == nullptr) {  // no context on this thread yet: the lookup makes the primary one current
+    void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_vs_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev].store(p, std::memory_order_release);
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
   }
-  *out = p;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchSlot& slot = g_scratch_slot[dev];
+  if (slot.ctx_id != id || slot.addr == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_vs_scratch);
+    if (e != cudaSuccess) return e;
+    slot.addr = p;
+    slot.ctx_id = id;
+  }
+  *out = slot.addr;
   return cudaSuccess;
 }
 

@@ -232,3 +232,68 @@ def test_maximum_sequence_length(cuda_device):
     Or, lr = oracle.attn_rows(Qb, Kb, Vb, 0, rows, vi, vc, si, sc)
     compare_rows(dev_to_f64(O)[rows, 0], Or, lse.cpu().numpy().astype(np.float64)[0, rows], lr,
                  what="N = 2^22")
+
+
+def _unit_plan(N, v, s, p):
+    """The attention kernel's per-unit choice for the 256-row unit at pair p,
+    restated from the plan's definition (key blocks on block-diagonals touched
+    by an offset, 128-column chunks of the columns <= the unit's last row):
+    returns (vertical chunks, slash key blocks, dense key blocks)."""
+    T = (N + 127) // 128
+    touched = set()
+    for o in s:
+        touched.add(int(o) >> 7)
+        if (int(o) & 127) and (int(o) >> 7) + 1 < T:
+            touched.add((int(o) >> 7) + 1)
+    d1 = touched | {t + 1 for t in touched}
+    last_b = min(2 * p + 1, T - 1)
+    nslash = sum(1 for x in d1 if 2 * p + 1 - last_b <= x <= 2 * p + 1)
+    nvc = (int(np.count_nonzero(np.asarray(v) <= min(256 * p + 255, N - 1))) + 127) // 128
+    return nvc, nslash, last_b + 1
+
+
+@pytest.mark.slow
+def test_split_path_many_vertical_chunks(cuda_device):
+    # N = 32768: the last units stream 64-128 vertical chunks each (split
+    # mode), the chunks at the diagonal straddle it (columns above some rows
+    # of the unit), and many columns also lie on selected diagonals (counted
+    # once).  Run with the plan-only workspace (row gathers) and with room
+    # for the packed rows (tile loads): identical outputs, checked against
+    # the oracle on the last two units' rows and sampled rows of every head.
+    from vs_testutil import sample_rows
+    N, d, Hq, Hkv = 32768, 128, 4, 2
+    rng = np.random.default_rng(31)
+    Qb, Kb, Vb = gen_qkv(32, N, Hq, Hkv, d, 500000.0)
+    v_sets = [np.sort(rng.choice(N, 9000, replace=False)),
+              np.arange(0, N, 4)[:8200],
+              np.sort(rng.choice(N, 16384, replace=False)),
+              np.sort(rng.choice(np.arange(3 * N // 4, N), 8192, replace=False))]
+    s_sets = [np.concatenate([np.arange(0, 50), [300, 1000, 5000]]),
+              np.concatenate([np.arange(0, 64), [127, 128, 129]]),
+              np.array([0, 1, 2]),
+              np.concatenate([np.arange(0, 10), [20000]])]
+    P = (N // 128 + 1) // 2
+    for v, s in zip(v_sets, s_sets):
+        for p in (P - 1, P - 2):
+            nvc, nslash, ndense = _unit_plan(N, v, s, p)
+            assert nvc + nslash < ndense and (p < P - 1 or nvc >= 64), (nvc, nslash, ndense)
+        assert np.intersect1d(v, N - 1 - s).size > 0  # a column on a selected diagonal
+    vi, vc = sets_to_rows(v_sets)
+    si, sc = sets_to_rows(s_sets)
+    Q, K, V = (bf16_to_dev(x) for x in (Qb, Kb, Vb))
+    args = [torch.from_numpy(x).cuda() for x in (vi, vc, si, sc)]
+    outs = []
+    for nbytes in (vs.vs_attn_workspace_size(N, Hq, Hq, d),
+                   vs.vs_attn_workspace_size_ld(N, Hq, Hq, d, vi.shape[1])):
+        ws = vs.workspace(nbytes)
+        O, lse = vs.sparse_attention(Q, K, V, *args, ws=ws)
+        rc, flags = vs.vs_read_device_status(ws)
+        assert rc == vs.VS_OK and flags == 0
+        outs.append((O.clone(), lse.clone()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    Od = dev_to_f64(outs[1][0])
+    lsed = outs[1][1].cpu().numpy().astype(np.float64)
+    for h in range(Hq):
+        rows = np.union1d(np.arange(N - 512, N), sample_rows(N, v_sets[h], seed=h, n_random=1024))
+        Or, lr = oracle.attn_rows(Qb, Kb, Vb, h, rows, vi, vc, si, sc)
+        compare_rows(Od[rows, h], Or, lsed[h, rows], lr, what=f"many chunks head {h}")

@@ -169,6 +169,29 @@ def test_flashprefill_32k_workload_full_size(cuda_device):
                      what=f"flashprefill_32k head {h}")
 
 
+@pytest.mark.slow
+def test_flashprefill_128k_workload_full_size(cuda_device):
+    # the bench's block workload itself: 32 query heads over 8 KV heads,
+    # N = 131072 (1024 query blocks); bit-exact kept-block masks for every
+    # head, then the block-sparse rows of every head sampled against the
+    # oracle over the oracle's masks
+    from vs_testutil import sample_rows
+    from vs_workloads import BLOCK_WORKLOADS
+    w = BLOCK_WORKLOADS["flashprefill_128k"]
+    Qb, Kb, Vb = w.qkv()
+    ref, margin = oracle.block_select(Qb, Kb, w.alpha)
+    assert (margin > 1e-9).all(), margin
+    got = _gpu_mask(bf16_to_dev(Qb), bf16_to_dev(Kb), w.alpha)
+    assert np.array_equal(got, ref)
+    O, lse = _gpu_block_attn(Qb, Kb, Vb, ref)
+    Od = dev_to_f64(O)
+    lsed = lse.cpu().numpy().astype(np.float64)
+    for h in range(w.Hq):
+        rows = sample_rows(w.N, seed=40 + h, n_random=512)
+        Or, lr = oracle.attn_block_rows(Qb, Kb, Vb, h, rows, ref)
+        compare_rows(Od[rows, h], Or, lsed[h, rows], lr, what=f"flashprefill_128k head {h}")
+
+
 @pytest.mark.parametrize("N,d,Hq,Hkv,alpha", [(3000, 128, 8, 2, 0.3), (2100, 64, 2, 2, 0.15)])
 def test_block_select_fp32_inputs(N, d, Hq, Hkv, alpha, cuda_device):
     # fp32 Q/K (off the bf16 grid) through the same selection; the oracle

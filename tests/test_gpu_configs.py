@@ -40,7 +40,7 @@ def _oracle_select(w, lv, ls):
 
 
 @pytest.mark.parametrize("name", ["tiny_1k", "llama_8k", "llama_32k", "llama_128k",
-                                  "llama_128k_maxfrac", "llama_256k_indexer"])
+                                  "llama_128k_S", "llama_128k_maxfrac", "llama_256k_indexer"])
 def test_full_size_workload(name, cuda_device):
     w = WORKLOADS[name]
     N, Hq, mode = w.N, w.Hq, w.select_mode_id

@@ -136,8 +136,9 @@ def test_maximum_row_length(cuda_device):
 @pytest.mark.parametrize("H,N", [(32, 131072), (8, 262144), (3, 5000)])
 def test_threshold_repeatable_bit_for_bit(H, N, cuda_device):
     # the fp64 mass sums have a fixed order (per-warp histograms, warp-order
-    # and rank-order merges): repeated calls give identical selections, with
-    # 4-, 16- and 2-CTA clusters (the three shapes below)
+    # and rank-order merges): repeated calls of one shape give identical
+    # selections; each of the three shapes below runs on its own cluster size
+    # (4, 16 and 2 CTAs), and the order differs from one size to another
     import torch
     rng = np.random.default_rng(N + H)
     s = torch.from_numpy((rng.standard_normal((H, N)) * 3.0).astype(np.float32)).cuda()

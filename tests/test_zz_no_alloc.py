@@ -2,9 +2,10 @@
 through the C ABI, against the workspace-based vs_sparse_attn_fwd.
 
 It serves callers that cannot allocate device memory (plain-C hosts without a
-memory manager, plug-ins inside engines that own the whole device pool).  Two
-calls in a row with different index sets check that the shared static scratch
-carries nothing over from the previous call.  Collected last on purpose."""
+memory manager, plug-ins inside engines that own the whole device pool).  Calls in a
+row with different index sets check that the shared static scratch carries
+nothing over from the previous call: the same index sets give the same bits
+before and after a call with other sets.  Collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -44,7 +45,8 @@ def test_static_scratch_matches_workspace_entry_point(cuda_device):
         vi, vc = vs.select(sv, vs.VS_SELECT_TOPK, w.k_v)
         si, sc = vs.select(ss, vs.VS_SELECT_TOPK, w.k_s)
         sets.append((vi, vc, si, sc))
-    for vi, vc, si, sc in sets:  # two calls in a row
+    outs = []
+    for vi, vc, si, sc in (sets[1], sets[0], sets[1]):  # three calls in a row
         O = torch.empty_like(Q)
         lse = torch.empty((w.Hq, w.N), dtype=torch.float32, device="cuda")
         assert _static_call(Q, K, V, vi, vc, si, sc, O, lse) == vs.VS_OK
@@ -53,6 +55,10 @@ def test_static_scratch_matches_workspace_entry_point(cuda_device):
         err = (O.float() - Oref.float()).abs()
         assert err.max().item() <= BF16_MAX_ABS and err.mean().item() <= BF16_MEAN_ABS
         assert torch.allclose(lse, lref, atol=1e-3, rtol=0)
+        outs.append((O, lse))
+    # the second index-set pair gives the same bits whether the scratch was
+    # last used by nothing or by the first pair: no state carries over
+    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
 
 
 def test_static_scratch_rejects_oversized_plans(cuda_device):
