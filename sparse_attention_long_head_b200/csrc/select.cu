@@ -14,9 +14,18 @@
 //     32-bit keys in shared memory.
 //   * Most-significant-digit radix searches (4 passes of 8 bits) find the
 //     exact boundary keys.  Per pass every CTA builds 256-bucket histograms
-//     of counts and, for the threshold rule, of fp64 softmax mass; the cluster
+//     (counts, and for the threshold rule fp64 softmax mass); the cluster
 //     merges them through distributed shared memory, and every CTA takes the
 //     same decision from the same merged data.
+//   * The threshold rule keeps k = min(k_threshold, cap) entries, so its mass
+//     matters only when the top-cap entries already reach tau * Z.  The kernel
+//     takes Z in one pass (fixed-order fp64 sum), runs the count search for
+//     the cap, and sums the top-cap entries' mass; only when that reaches
+//     tau * Z does the mass search run, and then over the keys at or above
+//     the cap's boundary key alone (packed in index order into a short list
+//     when it fits): every key of the threshold's prefix is among them.  A
+//     key's mass is exp(s - s_max) in fp64 (Tang's table-driven method,
+//     exp64.cuh).
 //   * The mass histogram takes no fp64 atomics (shared-memory fp64 atomic
 //     adds cost more than half of this kernel's time when they were used,
 //     by measurement): each warp owns a private copy; lanes holding
@@ -25,19 +34,16 @@
 //     a plain read-modify-write (distinct groups touch distinct buckets).
 //     The CTA's histogram is the warps' copies added in warp order, so the
 //     whole sum is in a fixed order and the selection is deterministic.
-//   * The threshold rule walks the buckets from the top, accumulating mass
-//     until tau * Z is reached (Z = the total of the first pass's mass
-//     histogram); inside the final group of equal keys the count follows from
-//     their common mass.  The top-cap boundary is searched in the same passes,
-//     so a capped head needs no second search.
 //   * FlashPrefill's max-based rule (summary page, section 2B: keep what
 //     scores at least alpha times the maximum, no sort and no cumulative sum)
 //     is one counting pass after the maximum; the kept entries are all keys
 //     at or above a boundary, so unless the cap binds no search runs at all.
-//   * A last pass writes the kept indices in ascending order (index-ordered
-//     compaction across the cluster), then pads with -1.
+//   * A last pass writes the kept indices in ascending order: each warp takes
+//     a contiguous range, 32 consecutive keys per step (conflict-free
+//     shared-memory reads), and ballots place the kept ones; then -1 pads.
 #include <cooperative_groups.h>
 
+#include "exp64.cuh"
 #include "internal.h"
 
 namespace cg = cooperative_groups;
@@ -47,6 +53,8 @@ namespace vs {
 constexpr int kSelThreads = 1024;
 constexpr int kSelMaxCluster = 8;
 constexpr int kSelCacheKeys = 32768;  // 128 KB of keys per CTA
+// dynamic shared memory per CTA (the static part, ~13 KB, stays under the 227 KB limit)
+constexpr size_t kSelMaxDynSmem = 208 * 1024;
 
 // Order-preserving key: larger key = earlier in (score desc); NaN -> 0
 // (after everything, including -inf); -0.0 is folded onto +0.0.
@@ -73,6 +81,7 @@ struct SelArgs {
   int32_t* count;
   int* status;
   int chunk;
+  int list_cap;  // threshold rule: room for the mass search's candidate keys (after wmass)
 };
 
 struct SelShared {
@@ -88,16 +97,27 @@ struct SelShared {
   int bstar_c, bstar_t;
   uint32_t cabove_c, cabove_t, eqcnt_t;
   double mabove_t, target;
+  double zpart, mpart;      // this CTA's share of Z, of the top-cap mass
+  double exp_tab[32];       // 2^(j/32) for exp_nonpos
   int wred_i[32];
   double wred_d[32];
-  int scan_a[kSelThreads];
-  int scan_b[kSelThreads];
+  uint32_t wg[32], we[32];  // per-warp counts of the compaction
 };
 
-__device__ __forceinline__ double pmass(uint32_t key, uint32_t kmax, double smax) {
+// Softmax mass of a key relative to the maximum: 1 for the maximum, 0 for
+// NaN.  The mass sums use exp_nonpos (relative error <= 1e-14, masses below
+// e^-700 dropped: negligible against sums of at least 1); the "p > 0" test
+// of tau = 1 uses the library exp, whose results reach down to the fp64
+// subnormals.
+__device__ __forceinline__ double pmass(uint32_t key, uint32_t kmax, double smax, const double* tab) {
   if (key == kmax) return 1.0;
   if (key == 0u) return 0.0;
-  return exp(static_cast<double>(fkey_inv(key)) - smax);
+  return exp_nonpos(static_cast<double>(fkey_inv(key)) - smax, tab);
+}
+__device__ __forceinline__ bool pmass_positive(uint32_t key, uint32_t kmax, double smax) {
+  if (key == kmax) return true;
+  if (key == 0u) return false;
+  return exp(static_cast<double>(fkey_inv(key)) - smax) > 0.0;
 }
 
 template <typename T, typename Op>
@@ -108,22 +128,6 @@ __device__ __forceinline__ T block_reduce(T v, T* wred, Op op) {
   __syncthreads();
   T r = wred[0];
   for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = op(r, wred[w]);
-  __syncthreads();
-  return r;
-}
-
-// Exclusive prefix sum over the block (int), returns this thread's prefix.
-__device__ __forceinline__ int block_excl_scan(int v, int* buf) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  buf[tid] = v;
-  __syncthreads();
-  for (int off = 1; off < nt; off <<= 1) {
-    int x = tid >= off ? buf[tid - off] : 0;
-    __syncthreads();
-    buf[tid] += x;
-    __syncthreads();
-  }
-  int r = buf[tid] - v;
   __syncthreads();
   return r;
 }
@@ -156,14 +160,19 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   const int tid = threadIdx.x, nt = blockDim.x;
   extern __shared__ uint32_t skeys[];
   __shared__ SelShared sh;
-  // per-warp mass histograms [warp][256], after the key cache (threshold rule only)
+  // per-warp mass histograms [warp][256], after the key cache (threshold rule
+  // only), then the candidate keys of the mass search
   double* wmass = reinterpret_cast<double*>(skeys + (CACHE ? (a.chunk + 1) / 2 * 2 : 0));
+  uint32_t* clist = reinterpret_cast<uint32_t*>(wmass + (kSelThreads / 32) * 256);
+  int ncand = 0;          // candidate keys of this CTA
+  bool use_list = false;  // the mass search reads clist (else every key, filtered)
 
   const float* row = a.scores + (int64_t)h * a.ld;
   const int lo = rank * a.chunk;
   const int n = max(0, min(a.N, lo + a.chunk) - lo);
   auto key_at = [&](int e) -> uint32_t { return CACHE ? skeys[e] : fkey(__ldg(row + lo + e)); };
 
+  if (tid < 32) sh.exp_tab[tid] = exp2((double)tid / 32.0);  // read after the cluster barrier below
   // ---- keys and the cluster-wide maximum key
   uint32_t lmax = 0;
   for (int e = tid; e < n; e += nt) {
@@ -179,17 +188,20 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   for (int r = 0; r < C; ++r) kmax = max(kmax, *cl.map_shared_rank(&sh.kmax, r));
   const double smax = static_cast<double>(fkey_inv(kmax));
 
-  // Two most-significant-digit radix searches share the passes over the keys:
-  //   count path: the key of the k-th entry (k = the top-k budget or the cap);
-  //   mass path (threshold rule): the key where the running softmax mass in
-  //     descending order reaches tau * Z; Z is the total of pass 0's mass
-  //     histogram, so it needs no pass of its own.
-  // The threshold result is used when it keeps at most `cap` entries, else the
-  // count path's top-cap result (k = min(k_threshold, cap)).
+  // Selection rules:
+  //   top-k: the count search for k;
+  //   max-based: one counting pass, the count search only if the cap binds;
+  //   threshold (tau < 1): k = min(k_threshold, cap), and the mass decides
+  //     only when it keeps at most `cap` entries.  So Z comes first (one pass,
+  //     a fixed-order sum), then the count search for the cap, then the mass
+  //     of the top-cap entries; only when that reaches tau * Z does the mass
+  //     search run, and only over the keys at or above the cap's boundary key
+  //     (every key of the threshold's prefix is among them).
   int k_count = a.k_or_cap;
-  bool use_mass = false;
+  bool thr = false;              // threshold rule with tau < 1 and a non-NaN maximum
   bool search = true;            // false: the kept set is every key >= kmin_kept
   uint32_t kmin_kept = 0xFFFFFFFFu;
+  const double* tab = sh.exp_tab;
   if (a.mode == VS_SELECT_MAXFRAC) {
     // keep r iff key_r == kmax or (double)s_r - s_max >= log(alpha); NaN
     // (key 0) never.  The test is monotone in the key, so the kept entries
@@ -229,7 +241,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
       k_count = 1;
     } else if (a.tau >= 1.0) {  // keep every entry with p > 0
       uint32_t c = 0;
-      for (int e = tid; e < n; e += nt) c += pmass(key_at(e), kmax, smax) > 0.0 ? 1u : 0u;
+      for (int e = tid; e < n; e += nt) c += pmass_positive(key_at(e), kmax, smax) ? 1u : 0u;
       c = static_cast<uint32_t>(block_reduce<int>(static_cast<int>(c), sh.wred_i,
                                                   [](int x, int y) { return x + y; }));
       if (tid == 0) sh.npos = c;
@@ -238,173 +250,205 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
       for (int r = 0; r < C; ++r) tot += static_cast<int>(*cl.map_shared_rank(&sh.npos, r));
       k_count = min(max(tot, 1), a.k_or_cap);
     } else {
-      use_mass = true;
+      thr = true;
     }
+  }
+  double target = 0.0;  // tau * Z
+  if (thr) {
+    // Z: per-thread partial sums over a fixed stride, a fixed tree over the
+    // block, the CTAs' shares added in rank order
+    double zp = 0.0;
+    for (int e = tid; e < n; e += nt) zp += pmass(key_at(e), kmax, smax, tab);
+    zp = block_reduce<double>(zp, sh.wred_d, [](double x, double y) { return x + y; });
+    if (tid == 0) sh.zpart = zp;
+    cl.sync();
+    double z = 0.0;
+    for (int r = 0; r < C; ++r) z += *cl.map_shared_rank(&sh.zpart, r);
+    target = a.tau * z;
   }
 
+  // Most-significant-digit radix search (4 passes of 8 bits).  Count path:
+  // the key of the k_count-th entry.  Mass path: the key where the running
+  // mass, in descending key order over the keys >= floor_key, reaches
+  // `target`.  Per pass every CTA builds 256-bucket histograms, the cluster
+  // merges them through DSMEM and every CTA takes the same decision.
   uint32_t pf_c = 0, pm_c = 0, cab_c = 0;            // count path
   uint32_t pf_t = 0, pm_t = 0, cab_t = 0, eq_t = 0;  // mass path
-  double mab_t = 0.0, target = 0.0;
+  double mab_t = 0.0;
   int buf = 0;
-  for (int pass = 0; pass < (search ? 4 : 0); ++pass) {
-    const int shift = 24 - 8 * pass;
-    if (tid < 256) {
-      sh.cnt_c[buf][tid] = 0;
-      sh.cnt_t[buf][tid] = 0;
-    }
-    if (use_mass)
-      for (int i = tid; i < (kSelThreads / 32) * 256; i += nt) wmass[i] = 0.0;
-    __syncthreads();
-    // Count path: run-length aggregation (keys of a pass often fall in one
-    // bucket, so a thread accumulates while its bucket repeats and flushes on
-    // change; the final flush is reduced across the warp when all lanes agree).
-    int cur_c = -1;
-    uint32_t rc_c = 0;
-    for (int e = tid; e < n; e += nt) {
-      const uint32_t k = key_at(e);
-      if ((k & pm_c) == pf_c) {
-        const int dg = (k >> shift) & 255;
-        if (dg != cur_c) {
-          if (cur_c >= 0) atomicAdd(&sh.cnt_c[buf][cur_c], rc_c);
-          cur_c = dg;
-          rc_c = 0;
-        }
-        ++rc_c;
+  auto radix = [&](bool do_count, bool do_mass, uint32_t floor_key) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      if (tid < 256) {
+        sh.cnt_c[buf][tid] = 0;
+        sh.cnt_t[buf][tid] = 0;
       }
-    }
-    __syncwarp();
-    {
-      const int c0 = __shfl_sync(0xffffffffu, cur_c, 0);
-      if (__all_sync(0xffffffffu, cur_c == c0) && c0 >= 0) {
-        const uint32_t r = __reduce_add_sync(0xffffffffu, rc_c);
-        if ((tid & 31) == 0) atomicAdd(&sh.cnt_c[buf][c0], r);
-      } else if (cur_c >= 0) {
-        atomicAdd(&sh.cnt_c[buf][cur_c], rc_c);
-      }
-    }
-    // Mass path: a warp takes 32 consecutive keys per step (warp-uniform trip
-    // count); lanes with equal digits form a group, whose lowest lane adds the
-    // group's count (shared atomic, integer) and mass (the warp's own
-    // histogram, plain add: the groups' digits differ).
-    if (use_mass) {
-      const int lane = tid & 31;
-      double* wm = wmass + (tid >> 5) * 256;
-      for (int base = tid - lane; base < n; base += nt) {
-        const int e = base + lane;
-        int dg = 256;  // 256: not in the searched prefix (or past the end)
-        double m = 0.0;
-        if (e < n) {
+      if (do_mass)
+        for (int i = tid; i < (kSelThreads / 32) * 256; i += nt) wmass[i] = 0.0;
+      __syncthreads();
+      if (do_count) {
+        // run-length aggregation (keys of a pass often fall in one bucket, so
+        // a thread accumulates while its bucket repeats and flushes on
+        // change; the final flush is reduced across the warp when all lanes
+        // agree)
+        int cur_c = -1;
+        uint32_t rc_c = 0;
+        for (int e = tid; e < n; e += nt) {
           const uint32_t k = key_at(e);
-          if ((k & pm_t) == pf_t) {
-            dg = (k >> shift) & 255;
-            m = pmass(k, kmax, smax);
+          if ((k & pm_c) == pf_c) {
+            const int dg = (k >> shift) & 255;
+            if (dg != cur_c) {
+              if (cur_c >= 0) atomicAdd(&sh.cnt_c[buf][cur_c], rc_c);
+              cur_c = dg;
+              rc_c = 0;
+            }
+            ++rc_c;
           }
         }
-        if (__all_sync(0xffffffffu, dg == __shfl_sync(0xffffffffu, dg, 0))) {
-          // one digit across the warp (the usual case in the first pass)
-          if (dg < 256) {
-            for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
-            if (lane == 0) {
-              atomicAdd(&sh.cnt_t[buf][dg], 32u);
-              wm[dg] += m;
+        __syncwarp();
+        const int c0 = __shfl_sync(0xffffffffu, cur_c, 0);
+        if (__all_sync(0xffffffffu, cur_c == c0) && c0 >= 0) {
+          const uint32_t r = __reduce_add_sync(0xffffffffu, rc_c);
+          if ((tid & 31) == 0) atomicAdd(&sh.cnt_c[buf][c0], r);
+        } else if (cur_c >= 0) {
+          atomicAdd(&sh.cnt_c[buf][cur_c], rc_c);
+        }
+      }
+      // Mass path: a warp takes 32 consecutive keys per step (warp-uniform
+      // trip count); lanes with equal digits form a group, whose lowest lane
+      // adds the group's count (shared atomic, integer) and mass (the warp's
+      // own histogram, plain add: the groups' digits differ).
+      if (do_mass) {
+        const int lane = tid & 31;
+        double* wm = wmass + (tid >> 5) * 256;
+        const int mn = use_list ? ncand : n;
+        for (int base = tid - lane; base < mn; base += nt) {
+          const int e = base + lane;
+          int dg = 256;  // 256: not in the searched prefix (or past the end)
+          double m = 0.0;
+          if (e < mn) {
+            const uint32_t k = use_list ? clist[e] : key_at(e);
+            if (k >= floor_key && (k & pm_t) == pf_t) {
+              dg = (k >> shift) & 255;
+              m = pmass(k, kmax, smax, tab);
             }
           }
-          continue;
+          if (__all_sync(0xffffffffu, dg == __shfl_sync(0xffffffffu, dg, 0))) {
+            if (dg < 256) {  // one digit across the warp
+              for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
+              if (lane == 0) {
+                atomicAdd(&sh.cnt_t[buf][dg], 32u);
+                wm[dg] += m;
+              }
+            }
+            continue;
+          }
+          const unsigned peers = __match_any_sync(0xffffffffu, dg);
+          const int gsize = __popc(peers);
+          const int gmax = __reduce_max_sync(0xffffffffu, (unsigned)gsize);
+          const int steps = 32 - __clz(gmax - 1);  // ceil(log2(gmax)); 0 for gmax = 1
+          m = group_sum(peers, m, steps);
+          if (dg < 256 && (peers & ((1u << lane) - 1u)) == 0) {
+            atomicAdd(&sh.cnt_t[buf][dg], (uint32_t)gsize);
+            wm[dg] += m;
+          }
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, dg);
-        const int gsize = __popc(peers);
-        const int gmax = __reduce_max_sync(0xffffffffu, (unsigned)gsize);
-        const int steps = 32 - __clz(gmax - 1);  // ceil(log2(gmax)); 0 for gmax = 1
-        m = group_sum(peers, m, steps);
-        if (dg < 256 && (peers & ((1u << lane) - 1u)) == 0) {
-          atomicAdd(&sh.cnt_t[buf][dg], (uint32_t)gsize);
-          wm[dg] += m;
+        __syncthreads();
+        if (tid < 256) {  // the CTA's histogram: the warps' copies in warp order
+          double t = 0.0;
+          for (int w = 0; w < kSelThreads / 32; ++w) t += wmass[w * 256 + tid];
+          sh.mass_t[buf][tid] = t;
         }
+      }
+      cl.sync();
+      if (tid < 256) {  // merge the cluster's histograms (same order in every CTA)
+        uint32_t cc = 0, ct = 0;
+        double mt = 0.0;
+        for (int r = 0; r < C; ++r) {
+          if (do_count) cc += cl.map_shared_rank(&sh.cnt_c[buf][0], r)[tid];
+          if (do_mass) {
+            ct += cl.map_shared_rank(&sh.cnt_t[buf][0], r)[tid];
+            mt += cl.map_shared_rank(&sh.mass_t[buf][0], r)[tid];
+          }
+        }
+        sh.tot_cc[tid] = cc;
+        sh.tot_ct[tid] = ct;
+        sh.tot_mt[tid] = mt;
       }
       __syncthreads();
-      if (tid < 256) {  // the CTA's histogram: the warps' copies in warp order
-        double t = 0.0;
-        for (int w = 0; w < kSelThreads / 32; ++w) t += wmass[w * 256 + tid];
-        sh.mass_t[buf][tid] = t;
-      }
-    }
-    cl.sync();
-    if (tid < 256) {  // merge the cluster's histograms (same order in every CTA)
-      uint32_t cc = 0, ct = 0;
-      double mt = 0.0;
-      for (int r = 0; r < C; ++r) {
-        cc += cl.map_shared_rank(&sh.cnt_c[buf][0], r)[tid];
-        if (use_mass) {
-          ct += cl.map_shared_rank(&sh.cnt_t[buf][0], r)[tid];
-          mt += cl.map_shared_rank(&sh.mass_t[buf][0], r)[tid];
+      if (do_count && tid < 32) {
+        // count path: the first bucket from the top at which the running
+        // count reaches k_count.  Lane l holds buckets 255 - 8 l .. 248 - 8 l.
+        const int lane = tid;
+        uint32_t c[8], tsum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          c[j] = sh.tot_cc[255 - 8 * lane - j];
+          tsum += c[j];
+        }
+        uint32_t incl = tsum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, cab_c + incl >= (uint32_t)k_count);
+        if (hit && lane == __ffs(hit) - 1) {
+          uint32_t ca = cab_c + incl - tsum;
+          int bs = -1;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (bs < 0 && c[j] != 0) {
+              if (ca + c[j] >= (uint32_t)k_count) bs = 255 - 8 * lane - j;
+              else ca += c[j];
+            }
+          }
+          sh.bstar_c = bs;
+          sh.cabove_c = ca;
         }
       }
-      sh.tot_cc[tid] = cc;
-      sh.tot_ct[tid] = ct;
-      sh.tot_mt[tid] = mt;
-    }
-    __syncthreads();
-    if (tid == 0) {  // count path: first bucket from the top reaching k_count
-      int bs = -1;
-      uint32_t ca = cab_c;
-      for (int b = 255; b >= 0; --b) {
-        const uint32_t c = sh.tot_cc[b];
-        if (c == 0) continue;
-        if (ca + c >= (uint32_t)k_count) {
-          bs = b;
-          break;
+      if (do_mass && tid == 32) {  // mass path: first bucket reaching the target
+        int bs = -1, last_nonempty = -1;
+        uint32_t ca = cab_t;
+        double ma = mab_t;
+        for (int b = 255; b >= 0; --b) {
+          const uint32_t c = sh.tot_ct[b];
+          if (c == 0) continue;
+          last_nonempty = b;
+          if (ma + sh.tot_mt[b] >= target) {
+            bs = b;
+            break;
+          }
+          ca += c;
+          ma += sh.tot_mt[b];
         }
-        ca += c;
-      }
-      sh.bstar_c = bs;
-      sh.cabove_c = ca;
-    }
-    if (use_mass && tid == 32) {  // mass path: first bucket reaching tau * Z
-      double tg = target;
-      if (pass == 0) {
-        double z = 0.0;
-        for (int b = 255; b >= 0; --b) z += sh.tot_mt[b];
-        tg = a.tau * z;
-        sh.target = tg;
-      }
-      int bs = -1, last_nonempty = -1;
-      uint32_t ca = cab_t;
-      double ma = mab_t;
-      for (int b = 255; b >= 0; --b) {
-        const uint32_t c = sh.tot_ct[b];
-        if (c == 0) continue;
-        last_nonempty = b;
-        if (ma + sh.tot_mt[b] >= tg) {
-          bs = b;
-          break;
+        if (bs < 0) {  // rounding left the total just short: take the last group
+          bs = last_nonempty;
+          ca -= sh.tot_ct[bs];
+          ma -= sh.tot_mt[bs];
         }
-        ca += c;
-        ma += sh.tot_mt[b];
+        sh.bstar_t = bs;
+        sh.cabove_t = ca;
+        sh.mabove_t = ma;
+        sh.eqcnt_t = sh.tot_ct[bs];
       }
-      if (bs < 0) {  // rounding left the total just short: take the last group
-        bs = last_nonempty;
-        ca -= sh.tot_ct[bs];
-        ma -= sh.tot_mt[bs];
+      __syncthreads();
+      if (do_count) {
+        pf_c |= static_cast<uint32_t>(sh.bstar_c) << shift;
+        pm_c |= 255u << shift;
+        cab_c = sh.cabove_c;
       }
-      sh.bstar_t = bs;
-      sh.cabove_t = ca;
-      sh.mabove_t = ma;
-      sh.eqcnt_t = sh.tot_ct[bs];
+      if (do_mass) {
+        pf_t |= static_cast<uint32_t>(sh.bstar_t) << shift;
+        pm_t |= 255u << shift;
+        cab_t = sh.cabove_t;
+        mab_t = sh.mabove_t;
+        eq_t = sh.eqcnt_t;
+      }
+      buf ^= 1;
     }
-    __syncthreads();
-    pf_c |= static_cast<uint32_t>(sh.bstar_c) << shift;
-    pm_c |= 255u << shift;
-    cab_c = sh.cabove_c;
-    if (use_mass) {
-      if (pass == 0) target = sh.target;
-      pf_t |= static_cast<uint32_t>(sh.bstar_t) << shift;
-      pm_t |= 255u << shift;
-      cab_t = sh.cabove_t;
-      mab_t = sh.mabove_t;
-      eq_t = sh.eqcnt_t;
-    }
-    buf ^= 1;
-  }
+  };
+  if (search) radix(true, false, 0u);
   uint32_t T = pf_c;
   uint32_t cabove = cab_c;
   int k_target = k_count;
@@ -412,34 +456,103 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
     T = kmin_kept - 1u;
     cabove = static_cast<uint32_t>(k_count);
   }
-  if (use_mass) {
-    // within the final group of equal keys every entry has the same mass
-    const double pstar = pmass(pf_t, kmax, smax);
-    double mm = pstar > 0.0 ? ceil((target - mab_t) / pstar) : static_cast<double>(eq_t);
-    mm = fmin(fmax(mm, 1.0), static_cast<double>(eq_t));
-    const int k_thr = static_cast<int>(cab_t) + static_cast<int>(mm);
-    if (k_thr <= a.k_or_cap) {
-      T = pf_t;
-      cabove = cab_t;
-      k_target = k_thr;
+  if (thr) {
+    // mass of the top-cap entries: the keys above the cap's boundary key,
+    // and as many copies of that key's mass as the cap keeps
+    double mp = 0.0;
+    for (int e = tid; e < n; e += nt) {
+      const uint32_t k = key_at(e);
+      if (k > pf_c) mp += pmass(k, kmax, smax, tab);
+    }
+    mp = block_reduce<double>(mp, sh.wred_d, [](double x, double y) { return x + y; });
+    if (tid == 0) sh.mpart = mp;
+    cl.sync();
+    double mcap = 0.0;
+    for (int r = 0; r < C; ++r) mcap += *cl.map_shared_rank(&sh.mpart, r);
+    mcap += static_cast<double>(k_count - static_cast<int>(cab_c)) * pmass(pf_c, kmax, smax, tab);
+    if (mcap >= target) {
+      // The threshold's prefix ends within the top-cap entries.  Their keys
+      // (>= the cap's boundary key; scattered over the row) are first packed
+      // in index order into a short list when it fits, so the four passes
+      // read only them.
+      {
+        const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+        const int wper = ((n + nw - 1) / nw + 31) / 32 * 32;
+        const int wb = min(n, warp * wper), wend = min(n, wb + wper);
+        uint32_t c = 0;
+        for (int base = wb; base < wend; base += 32) {
+          const int e = base + lane;
+          c += __popc(__ballot_sync(0xffffffffu, e < wend && key_at(e) >= pf_c));
+        }
+        if (lane == 0) sh.wg[warp] = c;
+        __syncthreads();
+        int off = 0;
+        for (int w = 0; w < nw; ++w) {
+          if (w < warp) off += static_cast<int>(sh.wg[w]);
+          ncand += static_cast<int>(sh.wg[w]);
+        }
+        use_list = ncand <= a.list_cap;
+        if (use_list) {
+          const unsigned lt = (1u << lane) - 1u;
+          for (int base = wb; base < wend; base += 32) {
+            const int e = base + lane;
+            const uint32_t k = e < wend ? key_at(e) : 0u;
+            const bool in = e < wend && k >= pf_c;
+            const unsigned m = __ballot_sync(0xffffffffu, in);
+            if (in) clist[off + __popc(m & lt)] = k;
+            off += __popc(m);
+          }
+        }
+        __syncthreads();
+      }
+      radix(false, true, pf_c);
+      // within the final group of equal keys every entry has the same mass
+      const double pstar = pmass(pf_t, kmax, smax, tab);
+      double mm = pstar > 0.0 ? ceil((target - mab_t) / pstar) : static_cast<double>(eq_t);
+      mm = fmin(fmax(mm, 1.0), static_cast<double>(eq_t));
+      const int k_thr = static_cast<int>(cab_t) + static_cast<int>(mm);
+      if (k_thr <= a.k_or_cap) {
+        T = pf_t;
+        cabove = cab_t;
+        k_target = k_thr;
+      }
     }
   }
   const int m_eq = k_target - static_cast<int>(cabove);  // equal keys to keep (smallest indices)
 
-  // ---- ascending compaction across the cluster
-  const int per = (n + nt - 1) / nt;
-  const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
-  int g = 0, q = 0;
-  for (int e = e0; e < e1; ++e) {
-    const uint32_t k = key_at(e);
-    g += k > T;
-    q += k == T;
+  // ---- ascending compaction across the cluster.  Warp w takes a contiguous
+  // range of keys, 32 consecutive keys per step (one per lane: conflict-free
+  // shared-memory reads); ballots give each kept key its place.
+  const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+  const int wper = ((n + nw - 1) / nw + 31) / 32 * 32;
+  const int wb = min(n, warp * wper), wend = min(n, wb + wper);
+  const unsigned lt = (1u << lane) - 1u;
+  {
+    uint32_t g = 0, q = 0;
+    for (int base = wb; base < wend; base += 32) {
+      const int e = base + lane;
+      const uint32_t k = e < wend ? key_at(e) : 0u;
+      g += __popc(__ballot_sync(0xffffffffu, e < wend && k > T));
+      q += __popc(__ballot_sync(0xffffffffu, e < wend && k == T));
+    }
+    if (lane == 0) {
+      sh.wg[warp] = g;
+      sh.we[warp] = q;
+    }
   }
-  const int G = block_excl_scan(g, sh.scan_a);
-  const int E = block_excl_scan(q, sh.scan_b);
-  if (tid == nt - 1) {
-    sh.gt = static_cast<uint32_t>(G + g);
-    sh.eq = static_cast<uint32_t>(E + q);
+  __syncthreads();
+  int G = 0, E = 0, Gt = 0, Et = 0;  // this warp's offsets; the CTA's totals
+  for (int w = 0; w < nw; ++w) {
+    if (w < warp) {
+      G += static_cast<int>(sh.wg[w]);
+      E += static_cast<int>(sh.we[w]);
+    }
+    Gt += static_cast<int>(sh.wg[w]);
+    Et += static_cast<int>(sh.we[w]);
+  }
+  if (tid == 0) {
+    sh.gt = static_cast<uint32_t>(Gt);
+    sh.eq = static_cast<uint32_t>(Et);
   }
   cl.sync();
   int eq_before = 0, sel_before = 0;
@@ -452,14 +565,17 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   int32_t* out = a.idx + (int64_t)h * a.ld_idx;
   int pos = sel_before + G + min(E, max(0, m_eq - eq_before));
   int eq_seen = eq_before + E;
-  for (int e = e0; e < e1; ++e) {
-    const uint32_t k = key_at(e);
-    if (k > T) {
-      out[pos++] = lo + e;
-    } else if (k == T) {
-      if (eq_seen < m_eq) out[pos++] = lo + e;
-      ++eq_seen;
-    }
+  for (int base = wb; base < wend; base += 32) {
+    const int e = base + lane;
+    const bool in = e < wend;
+    const uint32_t k = in ? key_at(e) : 0u;
+    const bool isg = in && k > T, ise = in && k == T;
+    const unsigned me = __ballot_sync(0xffffffffu, ise);
+    const bool keep = isg || (ise && eq_seen + __popc(me & lt) < m_eq);
+    const unsigned mk = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[pos + __popc(mk & lt)] = lo + e;
+    pos += __popc(mk);
+    eq_seen += __popc(me);
   }
   // pad [k, k_or_cap) with -1, split over the cluster
   for (int64_t t = (int64_t)k_target + rank * nt + tid; t < a.k_or_cap; t += (int64_t)C * nt) out[t] = -1;
@@ -482,6 +598,14 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
     if (cmin < C && H * C > sms && H * cmin <= sms) C = cmin;
   }
   const size_t mass_bytes = mode == VS_SELECT_THRESHOLD ? sizeof(double) * (kSelThreads / 32) * 256 : 0;
+  // Room for the threshold rule's candidate list: what is left of the
+  // dynamic shared memory, at most one entry per key of the CTA.
+  auto list_entries = [&](int chunk_, bool cache_) -> int {
+    if (mode != VS_SELECT_THRESHOLD) return 0;
+    const size_t used = (cache_ ? sizeof(uint32_t) * ((chunk_ + 1) / 2 * 2) : 0) + mass_bytes;
+    const size_t room = used < kSelMaxDynSmem ? (kSelMaxDynSmem - used) / sizeof(uint32_t) : 0;
+    return static_cast<int>(room < (size_t)chunk_ ? room : (size_t)chunk_);
+  };
   // Few heads leave most SMs idle: split long rows over 16-CTA clusters (a
   // non-portable size: used only when the device can place such a cluster).
   bool wide = C == kSelMaxCluster && H * kSelMaxCluster * 2 <= device_sm_count() &&
@@ -493,7 +617,8 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
     cudaLaunchConfig_t probe = {};
     probe.gridDim = dim3(16, H, 1);
     probe.blockDim = dim3(kSelThreads, 1, 1);
-    probe.dynamicSmemBytes = (cache16 ? sizeof(uint32_t) * ((chunk16 + 1) / 2 * 2) : 0) + mass_bytes;
+    probe.dynamicSmemBytes = (cache16 ? sizeof(uint32_t) * ((chunk16 + 1) / 2 * 2) : 0) + mass_bytes +
+                             sizeof(uint32_t) * list_entries(chunk16, cache16);
     cudaLaunchAttribute pa[1];
     pa[0].id = cudaLaunchAttributeClusterDimension;
     pa[0].val.clusterDim.x = 16;
@@ -515,11 +640,13 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
   if (wide) C = 16;
   const int chunk = (N + C - 1) / C;
   const bool cache = chunk <= kSelCacheKeys;
-  SelArgs a{scores, N, ld, mode, k_or_cap, tau, ln_alpha, idx, ld_idx, count, status, chunk};
+  const int list_cap = list_entries(chunk, cache);
+  SelArgs a{scores, N, ld, mode, k_or_cap, tau, ln_alpha, idx, ld_idx, count, status, chunk, list_cap};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, H, 1);
   cfg.blockDim = dim3(kSelThreads, 1, 1);
-  cfg.dynamicSmemBytes = (cache ? sizeof(uint32_t) * ((chunk + 1) / 2 * 2) : 0) + mass_bytes;
+  cfg.dynamicSmemBytes = (cache ? sizeof(uint32_t) * ((chunk + 1) / 2 * 2) : 0) + mass_bytes +
+                         sizeof(uint32_t) * list_cap;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
