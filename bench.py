@@ -224,6 +224,30 @@ def head_shard(Hq: int, Hkv: int, H_sel: int, world: int, rank: int):
     return q0, q1, kv0, kv1, int(q0 * s_per_q), int(q1 * s_per_q)
 
 
+def time_e2e(e2e_step, stream, flush, steps: int):
+    """Device time of `steps` end-to-end steps, as the kernel steps are timed:
+    one untimed warm-up step, then each timed step after an L2 flush written
+    outside its timed window.  Returns the per-step times in ms."""
+    import torch
+    e2e_step()
+    ts = []
+    for _ in range(max(1, steps)):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return ts
+
+
+E2E_PROTOCOL = ("mean of the timed steps, each after an L2 flush outside its timed window, "
+                "after one untimed warm-up step (the device step's protocol)")
+
+
 def whole_job_value(world: int, flops_per_rank: float, ms: float) -> float:
     """Aggregate effective TFLOP/s: every rank processes one replica of the layer in
     (at most) `ms`, so the job does world x flops in that time."""
@@ -613,16 +637,7 @@ def run_ours(args, w):
             stream.wait_stream(s_out)
             stream.wait_stream(cs[1])
 
-        ts = []
-        for it in range(3):
-            torch.cuda.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            e2e_step()
-            b.record(stream)
-            b.synchronize()
-            ts.append(a.elapsed_time(b))
+        ts = time_e2e(e2e_step, stream, flush, args.steps)
         # the pipelined result is the one-call result
         O_ref = O.clone()
         step(False)
@@ -630,10 +645,10 @@ def run_ours(args, w):
         if not torch.equal(O, O_ref):
             raise RuntimeError("pipelined end-to-end output differs from the one-call output")
         del O_ref
-        e2e_ms = max_over_ranks([float(np.min(ts[1:] if len(ts) > 1 else ts))], dev)[0]
+        e2e_ms = max_over_ranks([float(np.mean(ts))], dev)[0]
         e2e = {"value": round(job_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h),
+               "d2h_bytes_per_step": int(d2h), "protocol": E2E_PROTOCOL,
                "pipeline": "KV groups in the order of the shortest modelled copy-in / compute / "
                            "copy-out schedule (first and last split into heads): copy-in stream, "
                            "two alternating compute streams, copy-out stream"}
@@ -1104,16 +1119,7 @@ def run_batch(args, w):
             stream.wait_stream(s_out)
             stream.wait_stream(cs[1])
 
-        ts = []
-        for _ in range(3):
-            torch.cuda.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b_ = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            e2e_step()
-            b_.record(stream)
-            b_.synchronize()
-            ts.append(a.elapsed_time(b_))
+        ts = time_e2e(e2e_step, stream, flush, args.steps)
         for x in ws_att2:
             rc, flags = vs.vs_read_device_status(x)
             if rc != vs.VS_OK:
@@ -1124,10 +1130,10 @@ def run_batch(args, w):
         if not torch.equal(O, O_ref):
             raise RuntimeError("pipelined end-to-end output differs from the one-call output")
         del O_ref
-        e2e_ms = max_over_ranks([float(np.min(ts[1:]))], dev)[0]
+        e2e_ms = max_over_ranks([float(np.mean(ts))], dev)[0]
         e2e = {"value": round(whole_job_value(world, flops, e2e_ms), 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h),
+               "d2h_bytes_per_step": int(d2h), "protocol": E2E_PROTOCOL,
                "pipeline": f"{len(chunks)} chunks of consecutive sequences: copy-in stream, two "
                            "alternating compute streams (selects + one batched attention call per "
                            "chunk), copy-out stream"}
@@ -1327,16 +1333,7 @@ def run_blocks(args, w):
             stream.wait_stream(s_out)
             stream.wait_stream(cs[1])
 
-        ts = []
-        for _ in range(3):
-            torch.cuda.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b_ = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            e2e_step()
-            b_.record(stream)
-            b_.synchronize()
-            ts.append(a.elapsed_time(b_))
+        ts = time_e2e(e2e_step, stream, flush, args.steps)
         for x in ws2:
             rc, flags = vs.vs_read_device_status(x)
             if rc != vs.VS_OK:
@@ -1347,10 +1344,10 @@ def run_blocks(args, w):
         if not torch.equal(O, O_ref):
             raise RuntimeError("pipelined end-to-end output differs from the one-call output")
         del O_ref
-        e2e_ms = max_over_ranks([float(np.min(ts[1:]))], dev)[0]
+        e2e_ms = max_over_ranks([float(np.mean(ts))], dev)[0]
         e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h),
+               "d2h_bytes_per_step": int(d2h), "protocol": E2E_PROTOCOL,
                "pipeline": "KV groups in the order of the shortest modelled copy-in / compute / "
                            "copy-out schedule (first and last split into heads): copy-in stream, "
                            "two alternating compute streams (block discovery + block-sparse "
