@@ -267,6 +267,43 @@ vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, 
                                    size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * vs_block_select_varlen / vs_block_sparse_attn_fwd_varlen -- the block
+ * discovery and the block-sparse attention above for B sequences packed along
+ * the token axis (batched prefill; FlashPrefill summary page, sections 2A,
+ * 2B and 3, applied to each sequence on its own: blocks, probes and the
+ * alpha-times-best rule are per sequence, and a sequence attends only to
+ * itself).
+ *   total_tokens, cu_seqlens, max_seqlen  as for vs_sparse_attn_fwd_varlen
+ *            (cu_seqlens on the DEVICE; a malformed entry empties that
+ *            sequence and sets VS_DEVFLAG_BOUNDS).
+ *   mask / block_mask  uint32 [B][Hq][T][W] with T = ceil(max_seqlen / 128),
+ *            W = ceil(T / 32): sequence b's rows of head h at (b * Hq + h) * T;
+ *            vs_block_select_varlen writes rows I >= that sequence's block
+ *            count as zeros.  Each sequence's rows equal what vs_block_select
+ *            writes for that sequence alone (same arithmetic, same order).
+ *   O, lse   as for vs_sparse_attn_fwd_varlen (lse fp32 [Hq][total_tokens]).
+ *   ws       vs_block_select_workspace_size_varlen(B, max_seqlen, Hkv, d) and
+ *            vs_block_attn_workspace_size_varlen(B, max_seqlen, Hq) bytes,
+ *            256-byte aligned.
+ * Requires 1 <= max_seqlen <= 2^18; VS_ERR_UNSUPPORTED when the batch's
+ * per-(sequence, head) block lists would not fit 32-bit offsets.
+ */
+size_t vs_block_select_workspace_size_varlen(int B, int max_seqlen, int Hkv, int d);
+vs_status vs_block_select_varlen(const void* Q, const void* K, vs_dtype dtype, int total_tokens,
+                                 int B, const int32_t* cu_seqlens, int max_seqlen, int Hq,
+                                 int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                                 float softmax_scale, double alpha, uint32_t* mask, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream);
+size_t vs_block_attn_workspace_size_varlen(int B, int max_seqlen, int Hq);
+vs_status vs_block_sparse_attn_fwd_varlen(const void* Q, const void* K, const void* V,
+                                          vs_dtype dtype, int total_tokens, int B,
+                                          const int32_t* cu_seqlens, int max_seqlen, int Hq,
+                                          int Hkv, int d, int64_t q_stride_tok,
+                                          int64_t kv_stride_tok, float softmax_scale,
+                                          const uint32_t* block_mask, void* O, float* lse,
+                                          void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * vs_sparse_attn_fwd_static_scratch -- vs_sparse_attn_fwd without a
  * caller-provided workspace.  The summary pages have no counterpart to this
  * call; it exists for callers that cannot allocate device memory: plain-C

@@ -44,6 +44,8 @@ EXPORTS = (
     "vs_attn_aggregate", "vs_attn_workspace_size_varlen", "vs_sparse_attn_fwd_varlen",
     "vs_dense_attn_fwd_varlen", "vs_block_select_workspace_size", "vs_block_select",
     "vs_block_attn_workspace_size", "vs_block_sparse_attn_fwd", "vs_selftest_exp",
+    "vs_block_select_workspace_size_varlen", "vs_block_select_varlen",
+    "vs_block_attn_workspace_size_varlen", "vs_block_sparse_attn_fwd_varlen",
 )
 
 
@@ -105,6 +107,16 @@ def lib() -> ctypes.CDLL:
         L.vs_block_sparse_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I64, I64, F, P, P, P, P, Z,
                                                P]
         L.vs_block_sparse_attn_fwd.restype = I
+        L.vs_block_select_workspace_size_varlen.argtypes = [I, I, I, I]
+        L.vs_block_select_workspace_size_varlen.restype = Z
+        L.vs_block_select_varlen.argtypes = [P, P, I, I, I, P, I, I, I, I, I64, I64, F, D, P, P, Z,
+                                             P]
+        L.vs_block_select_varlen.restype = I
+        L.vs_block_attn_workspace_size_varlen.argtypes = [I, I, I]
+        L.vs_block_attn_workspace_size_varlen.restype = Z
+        L.vs_block_sparse_attn_fwd_varlen.argtypes = [P, P, P, I, I, I, P, I, I, I, I, I64, I64, F,
+                                                      P, P, P, P, Z, P]
+        L.vs_block_sparse_attn_fwd_varlen.restype = I
         L.vs_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
         L.vs_read_device_status.restype = I
         L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
@@ -275,6 +287,53 @@ def vs_block_sparse_attn_fwd(Q, K, V, mask, O, lse, ws, softmax_scale=0.0, strea
                                           Q.stride(0), K.stride(0), float(softmax_scale),
                                           _ptr(mask), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
                                           _stream(stream)), "vs_block_sparse_attn_fwd")
+
+
+def vs_block_select_workspace_size_varlen(B: int, max_seqlen: int, Hkv: int, d: int) -> int:
+    return int(lib().vs_block_select_workspace_size_varlen(B, max_seqlen, Hkv, d))
+
+
+def vs_block_attn_workspace_size_varlen(B: int, max_seqlen: int, Hq: int) -> int:
+    return int(lib().vs_block_attn_workspace_size_varlen(B, max_seqlen, Hq))
+
+
+def vs_block_select_varlen(Q, K, cu_seqlens, max_seqlen, alpha, mask, ws, softmax_scale=0.0,
+                           stream=None):
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    _check(lib().vs_block_select_varlen(
+        _ptr(Q), _ptr(K), _dtype(Q), T, B, _ptr(cu_seqlens), int(max_seqlen), Hq, Hkv, d,
+        Q.stride(0), K.stride(0), float(softmax_scale), float(alpha), _ptr(mask), _ptr(ws),
+        ws.numel(), _stream(stream)), "vs_block_select_varlen")
+
+
+def vs_block_sparse_attn_fwd_varlen(Q, K, V, cu_seqlens, max_seqlen, mask, O, lse, ws,
+                                    softmax_scale=0.0, stream=None):
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    _check(lib().vs_block_sparse_attn_fwd_varlen(
+        _ptr(Q), _ptr(K), _ptr(V), _dtype(Q), T, B, _ptr(cu_seqlens), int(max_seqlen), Hq, Hkv, d,
+        Q.stride(0), K.stride(0), float(softmax_scale), _ptr(mask), _ptr(O), _ptr(lse), _ptr(ws),
+        ws.numel(), _stream(stream)), "vs_block_sparse_attn_fwd_varlen")
+
+
+def block_prefill_varlen(Q, K, V, cu_seqlens, max_seqlen, alpha, stream=None):
+    """Batched block prefill: discovery then block-sparse attention per
+    sequence; returns (O, lse [Hq, total], mask [B, Hq, T, W])."""
+    total, Hq, d = Q.shape
+    B = cu_seqlens.numel() - 1
+    T = (int(max_seqlen) + 127) // 128
+    mask = torch.empty((B, Hq, T, (T + 31) // 32), dtype=torch.int32, device=Q.device)
+    ws = workspace(max(vs_block_select_workspace_size_varlen(B, max_seqlen, K.shape[1], d),
+                       vs_block_attn_workspace_size_varlen(B, max_seqlen, Hq)), Q.device)
+    vs_block_select_varlen(Q, K, cu_seqlens, max_seqlen, alpha, mask, ws, stream=stream)
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, total), dtype=torch.float32, device=Q.device)
+    vs_block_sparse_attn_fwd_varlen(Q, K, V, cu_seqlens, max_seqlen, mask, O, lse, ws,
+                                    stream=stream)
+    return O, lse, mask
 
 
 def block_prefill(Q, K, V, alpha, stream=None):

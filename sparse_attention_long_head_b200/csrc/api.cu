@@ -317,23 +317,34 @@ size_t vs_block_select_workspace_size(int N, int Hkv, int d) {
   return block_select_ws_bytes(N, Hkv, d);
 }
 
-vs_status vs_block_select(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
-                          int d, int64_t q_stride_tok, int64_t kv_stride_tok, float softmax_scale,
-                          double alpha, uint32_t* mask, void* ws, size_t ws_bytes,
-                          cudaStream_t stream) {
+size_t vs_block_select_workspace_size_varlen(int B, int max_seqlen, int Hkv, int d) {
+  if (B < 1 || max_seqlen < 1 || Hkv < 1 || d < 1) return kStatusBytes;
+  return block_select_ws_bytes(max_seqlen, B * Hkv, d);
+}
+
+static vs_status block_select_impl(const void* Q, const void* K, vs_dtype dtype, int N, int B,
+                                   int64_t total, const int32_t* cu, int Hq, int Hkv, int d,
+                                   int64_t q_stride_tok, int64_t kv_stride_tok,
+                                   float softmax_scale, double alpha, uint32_t* mask, void* ws,
+                                   size_t ws_bytes, cudaStream_t stream) {
   if (!mask) return VS_ERR_INVALID_ARG;
   vs_status st = check_attn_common(Q, K, K, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
                                    softmax_scale, mask);
   if (st != VS_OK) return st;
-  if (!(alpha > 0.0 && alpha <= 1.0)) return VS_ERR_INVALID_ARG;
+  if (!(alpha > 0.0 && alpha <= 1.0) || B < 1 || total < 1) return VS_ERR_INVALID_ARG;
   if (N > (1 << 18)) return VS_ERR_UNSUPPORTED;
-  if (!ws || ws_bytes < block_select_ws_bytes(N, Hkv, d) || !aligned(ws, 256))
+  // work items (sequence, query block, head) are counted in 32 bits
+  if ((int64_t)B * ((N + 127) / 128) * Hq >= ((int64_t)1 << 31)) return VS_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < block_select_ws_bytes(N, B * Hkv, d) || !aligned(ws, 256))
     return VS_ERR_WORKSPACE;
   BlockSelectArgs a;
   a.Q = Q;
   a.K = K;
   a.dtype = dtype;
   a.N = N;
+  a.B = B;
+  a.total = total;
+  a.cu_seqlens = cu;
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.d = d;
@@ -349,23 +360,50 @@ vs_status vs_block_select(const void* Q, const void* K, vs_dtype dtype, int N, i
   return launch_block_select(a) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
 }
 
+vs_status vs_block_select(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
+                          int d, int64_t q_stride_tok, int64_t kv_stride_tok, float softmax_scale,
+                          double alpha, uint32_t* mask, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  return block_select_impl(Q, K, dtype, N, 1, N, nullptr, Hq, Hkv, d, q_stride_tok,
+                           kv_stride_tok, softmax_scale, alpha, mask, ws, ws_bytes, stream);
+}
+
+vs_status vs_block_select_varlen(const void* Q, const void* K, vs_dtype dtype, int total_tokens,
+                                 int B, const int32_t* cu_seqlens, int max_seqlen, int Hq,
+                                 int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                                 float softmax_scale, double alpha, uint32_t* mask, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream) {
+  if (!cu_seqlens) return VS_ERR_INVALID_ARG;
+  return block_select_impl(Q, K, dtype, max_seqlen, B, total_tokens, cu_seqlens, Hq, Hkv, d,
+                           q_stride_tok, kv_stride_tok, softmax_scale, alpha, mask, ws, ws_bytes,
+                           stream);
+}
+
 size_t vs_block_attn_workspace_size(int N, int Hq) {
   if (N < 1 || Hq < 1) return kStatusBytes;
   return BlockPlanLayout::make(N, Hq).total;
 }
 
-vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype,
-                                   int N, int Hq, int Hkv, int d, int64_t q_stride_tok,
-                                   int64_t kv_stride_tok, float softmax_scale,
-                                   const uint32_t* block_mask, void* O, float* lse, void* ws,
-                                   size_t ws_bytes, cudaStream_t stream) {
+size_t vs_block_attn_workspace_size_varlen(int B, int max_seqlen, int Hq) {
+  if (B < 1 || max_seqlen < 1 || Hq < 1) return kStatusBytes;
+  return BlockPlanLayout::make(max_seqlen, B * Hq).total;
+}
+
+static vs_status block_attn_impl(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                 int N, int B, int64_t total, const int32_t* cu, int Hq, int Hkv,
+                                 int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                                 float softmax_scale, const uint32_t* block_mask, void* O,
+                                 float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (!block_mask) return VS_ERR_INVALID_ARG;
   vs_status st = check_attn_common(Q, K, V, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
                                    softmax_scale, O);
   if (st != VS_OK) return st;
+  if (B < 1 || total < 1) return VS_ERR_INVALID_ARG;
   if (dtype != VS_BF16 || N > (1 << 18)) return VS_ERR_UNSUPPORTED;
-  if (!ws || ws_bytes < BlockPlanLayout::make(N, Hq).total || !aligned(ws, 256))
-    return VS_ERR_WORKSPACE;
+  const BlockPlanLayout BL = BlockPlanLayout::make(N, B * Hq);
+  // per-pair list offsets of every (sequence, head) must fit the kernel's 32-bit index
+  if ((int64_t)B * Hq * BL.P * (BL.P + 1) >= ((int64_t)1 << 31)) return VS_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < BL.total || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
   AttnArgs a{};
   a.Q = Q;
   a.K = K;
@@ -377,9 +415,9 @@ vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, 
   a.Hkv = Hkv;
   a.d = d;
   a.H_sel = 1;
-  a.B = 1;
-  a.total = N;
-  a.cu_seqlens = nullptr;
+  a.B = B;
+  a.total = total;
+  a.cu_seqlens = cu;
   a.q_stride = q_stride_tok;
   a.kv_stride = kv_stride_tok;
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
@@ -393,6 +431,28 @@ vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, 
   if (cudaMemsetAsync(a.status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
   if (launch_block_plan(a) != cudaSuccess) return VS_ERR_CUDA;
   return launch_attn_tc(a, L) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
+vs_status vs_block_sparse_attn_fwd(const void* Q, const void* K, const void* V, vs_dtype dtype,
+                                   int N, int Hq, int Hkv, int d, int64_t q_stride_tok,
+                                   int64_t kv_stride_tok, float softmax_scale,
+                                   const uint32_t* block_mask, void* O, float* lse, void* ws,
+                                   size_t ws_bytes, cudaStream_t stream) {
+  return block_attn_impl(Q, K, V, dtype, N, 1, N, nullptr, Hq, Hkv, d, q_stride_tok,
+                         kv_stride_tok, softmax_scale, block_mask, O, lse, ws, ws_bytes, stream);
+}
+
+vs_status vs_block_sparse_attn_fwd_varlen(const void* Q, const void* K, const void* V,
+                                          vs_dtype dtype, int total_tokens, int B,
+                                          const int32_t* cu_seqlens, int max_seqlen, int Hq,
+                                          int Hkv, int d, int64_t q_stride_tok,
+                                          int64_t kv_stride_tok, float softmax_scale,
+                                          const uint32_t* block_mask, void* O, float* lse,
+                                          void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!cu_seqlens) return VS_ERR_INVALID_ARG;
+  return block_attn_impl(Q, K, V, dtype, max_seqlen, B, total_tokens, cu_seqlens, Hq, Hkv, d,
+                         q_stride_tok, kv_stride_tok, softmax_scale, block_mask, O, lse, ws,
+                         ws_bytes, stream);
 }
 
 vs_status vs_read_device_status(const void* ws, cudaStream_t stream, int* flags) {

@@ -313,11 +313,14 @@ __global__ void __launch_bounds__(32) block_plan_kernel(const uint32_t* mask, in
   if (lane == 0) bcnt[(int64_t)h * P + p] = base;
 }
 
+// A batch of B sequences has mask rows and plan slots per (sequence, query
+// head), b * Hq + h: the same kernel over B * Hq "heads".
 cudaError_t launch_block_plan(const AttnArgs& a) {
-  const BlockPlanLayout B = BlockPlanLayout::make(a.N, a.Hq);
+  const BlockPlanLayout B = BlockPlanLayout::make(a.N, a.B * a.Hq);
   int32_t* bcnt = reinterpret_cast<int32_t*>(static_cast<char*>(a.ws) + B.off_cnt);
   uint32_t* blist = reinterpret_cast<uint32_t*>(static_cast<char*>(a.ws) + B.off_list);
-  block_plan_kernel<<<dim3(B.P, a.Hq), 32, 0, a.stream>>>(a.block_mask, B.T, B.P, bcnt, blist);
+  block_plan_kernel<<<dim3(B.P, a.B * a.Hq), 32, 0, a.stream>>>(a.block_mask, B.T, B.P, bcnt,
+                                                                blist);
   return cudaGetLastError();
 }
 
@@ -411,9 +414,10 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& P, int u) {
     return ui;
   }
   if (MODE == kAttnBlock) {
+    const int64_t hb = (int64_t)bseq * P.Hq + ui.h;  // plan slot of (sequence, head)
     ui.mode = kModeBlock;
-    ui.n = P.bcnt[(int64_t)ui.h * P.P + ui.p];
-    ui.d1start = ui.h * P.P * (P.P + 1) + ui.p * (ui.p + 1);
+    ui.n = P.bcnt[hb * P.P + ui.p];
+    ui.d1start = (int)(hb * P.P * (P.P + 1) + (int64_t)ui.p * (ui.p + 1));
     return ui;
   }
   const int32_t* d1pref = P.pp.d1pref + (int64_t)ui.hs * P.L.d1pref_len;
@@ -1078,7 +1082,7 @@ static cudaError_t launch_tc_impl(const AttnArgs& a, const PlanLayout& L) {
   P.bcnt = nullptr;
   P.blist = nullptr;
   if (MODE == kAttnBlock) {
-    const BlockPlanLayout B = BlockPlanLayout::make(a.N, a.Hq);
+    const BlockPlanLayout B = BlockPlanLayout::make(a.N, a.B * a.Hq);
     P.bcnt = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.ws) + B.off_cnt);
     P.blist = reinterpret_cast<const uint32_t*>(static_cast<const char*>(a.ws) + B.off_list);
   }

@@ -103,25 +103,39 @@ __host__ __device__ __forceinline__ int64_t kbar_frag_off(int D, int Tp, int g, 
   return (((int64_t)g * (Tp / 16) + tile) * (D / 16) + ks) * 256 + j * 64 + lane * 2 + e;
 }
 
-__global__ void __launch_bounds__(128) block_mean_kernel(const void* K, int dtype, int N, int T,
-                                                         int d, int64_t kv_stride, double* kbar) {
-  const int J = blockIdx.x, g = blockIdx.y, Tp = gridDim.x;
-  const int64_t j0 = 128 * (int64_t)J, j1 = min((int64_t)N, j0 + 128);
+// One CTA per (key block J, KV head g, sequence b) of a batch packed along
+// the token axis (cu: B + 1 offsets; null for one sequence of N tokens);
+// the means of (b, g) are stored as those of KV head b * Hkv + g.  A
+// malformed entry gives an empty sequence (zero means) and the bounds flag.
+__global__ void __launch_bounds__(128) block_mean_kernel(const void* K, int dtype, int N, int d,
+                                                         int64_t kv_stride, const int32_t* cu,
+                                                         int64_t total, int* status,
+                                                         double* kbar) {
+  const int J = blockIdx.x, g = blockIdx.y, b = blockIdx.z, Tp = gridDim.x, Hkv = gridDim.y;
+  int64_t tok0;
+  int Nb;
+  if (!seq_range(cu, total, N, b, tok0, Nb) && J == 0 && g == 0 && threadIdx.x == 0)
+    atomicOr(status, VS_DEVFLAG_BOUNDS);
+  const int Tb = (Nb + 127) / 128;
+  const int64_t j0 = 128 * (int64_t)J, j1 = min((int64_t)Nb, j0 + 128);
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     double mean = 0.0;
-    if (J < T) {
+    if (J < Tb) {
       double acc = 0.0;
-      for (int64_t j = j0; j < j1; ++j) acc += load_kv(K, dtype, j * kv_stride + (int64_t)g * d + c);
+      for (int64_t j = j0; j < j1; ++j)
+        acc += load_kv(K, dtype, (tok0 + j) * kv_stride + (int64_t)g * d + c);
       mean = acc / (double)(j1 - j0);
     }
-    kbar[kbar_frag_off(d, Tp, g, J, c)] = mean;
+    kbar[kbar_frag_off(d, Tp, b * Hkv + g, J, c)] = mean;
   }
 }
 
 struct ScoreArgs {
   const void* Q;
   int dtype, N, Hq, Hkv, T, W, Tp, HC;  // HC: query heads per work item (1, 2 or 4)
-  int n_items, n_chunks;                // items: (query block, chunk of HC heads)
+  int n_items, n_chunks;                // items: (sequence, query block, chunk of HC heads)
+  const int32_t* cu;                    // sequence offsets (device) or null
+  int64_t total;
   int stages;                           // ring slots: 3, or 4 with two stage classes
   int64_t q_stride;
   double scale, alpha;
@@ -193,12 +207,22 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
   __syncthreads();
   const WaitCtx wc{a.wait_limit_ns, a.status, &abort_flag};
   const int esz = a.dtype == VS_BF16 ? 2 : 4;
-  auto item_rows = [&](int k, int& I, int& h0, int& np, int& nsq) {
-    I = a.T - 1 - k / a.n_chunks;
-    h0 = (k % a.n_chunks) * a.HC;
+  // Item k: sequence b = k / (T n_chunks), then query blocks from the last,
+  // heaviest first.  An item whose block lies past its sequence's end
+  // (valid = false) only writes zero mask rows.
+  auto item_rows = [&](int k, int& b, int64_t& tok0, bool& valid, int& I, int& h0, int& np,
+                       int& nsq) {
+    const int per_seq = a.T * a.n_chunks;
+    b = k / per_seq;
+    const int rem = k - b * per_seq;
+    I = a.T - 1 - rem / a.n_chunks;
+    h0 = (rem % a.n_chunks) * a.HC;
+    int Nb;
+    seq_range(a.cu, a.total, a.N, b, tok0, Nb);
+    valid = 128 * (int64_t)I < Nb;
     np = 0;
-    while (np < kProbes && 128 * (int64_t)I + kProbeStride * np < a.N) ++np;
-    nsq = (I + 16 * kTilesPerStage - 1) / (16 * kTilesPerStage);  // 0 for I = 0
+    while (valid && np < kProbes && 128 * (int64_t)I + kProbeStride * np < Nb) ++np;
+    nsq = valid ? (I + 16 * kTilesPerStage - 1) / (16 * kTilesPerStage) : 0;  // 0 for I = 0
   };
 
   // ------------------------------------------------------------- producer
@@ -214,10 +238,12 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
         bool w = lane == 0 ? mbar_wait(smem_u32(&pempty_bar), (it - 1) & 1, wc) : true;
         if (!__shfl_sync(0xffffffffu, (int)w, 0)) break;
       }
-      int I = 0, h0 = 0, np = 0, nsq = 0;
+      int I = 0, h0 = 0, np = 0, nsq = 0, bq = 0;
+      int64_t tq0 = 0;
+      bool valid = false;
       if (k < a.n_items) {
-        item_rows(k, I, h0, np, nsq);
-        if (I > 0) {
+        item_rows(k, bq, tq0, valid, I, h0, np, nsq);
+        if (valid && I > 0) {
           // Probe rows (the HC heads' D values are contiguous and 16-byte
           // aligned) in 16-byte pieces, eight per lane in flight, scattered
           // into fragment order; rows past the probes are zeros.
@@ -232,7 +258,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
               if (e < kProbes * pieces && p < np)
                 v[x] = __ldg(reinterpret_cast<const uint4*>(
                                  static_cast<const uint8_t*>(a.Q) +
-                                 ((128 * (int64_t)I + kProbeStride * p) * a.q_stride +
+                                 ((tq0 + 128 * (int64_t)I + kProbeStride * p) * a.q_stride +
                                   (int64_t)h0 * D) * esz) + e % pieces);
             }
 #pragma unroll
@@ -264,7 +290,8 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
       if (lane == 0) mbar_arrive(smem_u32(&pfull_bar));  // release: the fragments and the item
       if (k >= a.n_items) break;
       if (lane == 0) {
-        const double* src = a.kbar + (int64_t)(h0 / (a.Hq / a.Hkv)) * (a.Tp / 16) * kTileDoubles;
+        const double* src =
+            a.kbar + ((int64_t)bq * a.Hkv + h0 / (a.Hq / a.Hkv)) * (a.Tp / 16) * kTileDoubles;
         for (int q = 0; q < nsq; ++q, ++s) {
           const int slot = s % a.stages, use = s / a.stages;
           if (use > 0 && !mbar_wait(smem_u32(&empty_bar[slot]), (use - 1) & 1, wc)) {
@@ -302,16 +329,22 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
     if (!named_bar_and(1, kCons, ok)) break;
     const int k = item_slot;
     if (k >= a.n_items) break;
-    int I, h0, np, nsq;
-    item_rows(k, I, h0, np, nsq);
+    int I, h0, np, nsq, bq;
+    int64_t tq0;
+    bool valid;
+    item_rows(k, bq, tq0, valid, I, h0, np, nsq);
     const int sb = s0;
     s0 += nsq;
-    if (I == 0) {  // no earlier block: the diagonal alone
+    // the item's mask rows: heads h0 .. h0 + HC - 1 of sequence bq, block I
+    auto mask_row = [&](int x) {
+      return a.mask + (((int64_t)bq * a.Hq + h0 + x) * a.T + I) * a.W;
+    };
+    if (!valid || I == 0) {  // past the sequence's end: nothing; block 0: the diagonal alone
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&pempty_bar));
       for (int e = tid; e < a.HC * a.W; e += kCons) {
         const int x = e / a.W, w = e % a.W;
-        a.mask[((int64_t)(h0 + x) * a.T) * a.W + w] = w == 0 ? 1u : 0u;
+        mask_row(x)[w] = (valid && w == 0) ? 1u : 0u;
       }
       continue;
     }
@@ -517,7 +550,7 @@ __global__ void __launch_bounds__(kBsThreads, 1) block_score_kernel(const ScoreA
       for (int w = 1; w < kBsWarps; ++w) b = fmax(b, red[w][x]);
       const double thr = a.alpha * b;
       const double* sc = score + x * a.T;
-      uint32_t* out = a.mask + ((int64_t)(h0 + x) * a.T + I) * a.W;
+      uint32_t* out = mask_row(x);
       for (int w = warp; w < a.W; w += kBsWarps) {
         const int J = 32 * w + lane;
         const bool keep = J == I || (J < I && sc[J] >= thr);
@@ -545,9 +578,9 @@ cudaError_t launch_exp_selftest(const double* x, double* y, int n, cudaStream_t 
   return cudaGetLastError();
 }
 
-size_t block_select_ws_bytes(int N, int Hkv, int d) {
+size_t block_select_ws_bytes(int N, int B_Hkv, int d) {
   const int T = (N + 127) / 128, Tp = pad_blocks(T), sms = num_sms();
-  return kStatusBytes + align_up(sizeof(double) * (size_t)Hkv * Tp * d, 256) +
+  return kStatusBytes + align_up(sizeof(double) * (size_t)B_Hkv * Tp * d, 256) +
          sizeof(double) * (size_t)(sms > 0 ? sms : 1) * scratch_doubles_per_cta(Tp);
 }
 
@@ -561,9 +594,9 @@ cudaError_t launch_block_select(const BlockSelectArgs& a) {
   char* base = static_cast<char*>(a.ws);
   double* kbar = reinterpret_cast<double*>(base + kStatusBytes);
   double* scratch = reinterpret_cast<double*>(
-      base + kStatusBytes + align_up(sizeof(double) * (size_t)a.Hkv * Tp * a.d, 256));
-  block_mean_kernel<<<dim3(Tp, a.Hkv), 128, 0, a.stream>>>(a.K, a.dtype, a.N, T, a.d, a.kv_stride,
-                                                           kbar);
+      base + kStatusBytes + align_up(sizeof(double) * (size_t)a.B * a.Hkv * Tp * a.d, 256));
+  block_mean_kernel<<<dim3(Tp, a.Hkv, a.B), 128, 0, a.stream>>>(
+      a.K, a.dtype, a.N, a.d, a.kv_stride, a.cu_seqlens, a.total, static_cast<int*>(a.ws), kbar);
   ScoreArgs s;
   s.Q = a.Q;
   s.dtype = a.dtype;
@@ -575,7 +608,9 @@ cudaError_t launch_block_select(const BlockSelectArgs& a) {
   s.Tp = Tp;
   s.HC = HC;
   s.n_chunks = a.Hq / HC;
-  s.n_items = T * s.n_chunks;
+  s.n_items = a.B * T * s.n_chunks;
+  s.cu = a.cu_seqlens;
+  s.total = a.total;
   s.q_stride = a.q_stride;
   s.scale = a.scale;
   s.alpha = a.alpha;

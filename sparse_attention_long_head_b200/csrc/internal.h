@@ -206,14 +206,18 @@ struct AggArgs {
 struct BlockSelectArgs {
   const void* Q;
   const void* K;
-  int dtype, N, Hq, Hkv, d;
+  int dtype, N, Hq, Hkv, d;  // N: the longest sequence (the only one when B = 1)
+  int B;                     // sequences packed along the token axis
+  int64_t total;             // token rows of Q and K
+  const int32_t* cu_seqlens; // device [B + 1] or null
   int64_t q_stride, kv_stride;
   double scale, alpha;
-  uint32_t* mask;  // [Hq][T][W]
+  uint32_t* mask;  // [B][Hq][T][W], T and W of the longest sequence
   void* ws;        // status word, then the block means
   cudaStream_t stream;
 };
-size_t block_select_ws_bytes(int N, int Hkv, int d);
+// workspace of a batch: the block means of B * Hkv (sequence, KV head) pairs
+size_t block_select_ws_bytes(int N, int B_Hkv, int d);
 cudaError_t launch_block_select(const BlockSelectArgs& a);
 cudaError_t launch_exp_selftest(const double* x, double* y, int n, cudaStream_t stream);
 
