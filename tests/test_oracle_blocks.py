@@ -86,6 +86,46 @@ def test_closed_form_constant_blocks():
             assert np.array_equal(got[I], want), (alpha, I)
 
 
+def test_closed_form_probe_rows_and_ragged_probe_count():
+    # Which rows probe: only rows 128 I + 8 m (m = 0..15, below N) carry the
+    # probe queries -- q1 = e1 for even m, q2 = e2 for odd m -- every other
+    # row carries -e1, which would invert the preferences if it were read.
+    # Keys are constant per block, k_J = ln(a_J) e1 + ln(b_J) e2, so with
+    # scale 1 a q1 probe gives softmax weights a_J / sum a and a q2 probe
+    # b_J / sum b over J < I.  A full block has 8 probes of each kind: score
+    # (P1 + P2) / 2; the last block here holds 20 rows, i.e. probes m = 0,
+    # 1, 2 (two q1, one q2): score (2 P1 + P2) / 3.
+    T, d = 6, 4
+    N = 128 * (T - 1) + 20
+    a = np.array([3.0, 0.4, 1.2, 2.0, 0.7, 1.0])
+    b = np.array([0.2, 2.5, 1.0, 0.5, 3.0, 1.0])
+    K = np.zeros((N, 1, d), np.float32)
+    for J in range(T):
+        rows = slice(128 * J, min(N, 128 * J + 128))
+        K[rows, 0, 1] = np.log(a[J])
+        K[rows, 0, 2] = np.log(b[J])
+    Q = np.zeros((N, 1, d), np.float32)
+    Q[:, 0, 1] = -1.0
+    for I in range(T):
+        for m in range(16):
+            i = 128 * I + 8 * m
+            if i < N:
+                Q[i, 0, 1], Q[i, 0, 2] = (1.0, 0.0) if m % 2 == 0 else (0.0, 1.0)
+    for alpha in (0.3, 0.6, 0.85):
+        mask, margin = oracle.block_select(Q, K, alpha, scale=1.0)
+        assert margin[0] > 1e-6, alpha
+        got = _unpack(mask, T)[0]
+        for I in range(T):
+            want = np.zeros(T, bool)
+            want[I] = True
+            if I:
+                p1 = a[:I] / a[:I].sum()
+                p2 = b[:I] / b[:I].sum()
+                score = (2 * p1 + p2) / 3 if I == T - 1 else (p1 + p2) / 2
+                want[:I] = score >= alpha * score.max()
+            assert np.array_equal(got[I], want), (alpha, I)
+
+
 def test_alpha_limits_and_monotonicity():
     rng = np.random.default_rng(4)
     N = 1000
