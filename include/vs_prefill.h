@@ -376,6 +376,24 @@ vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N,
                             void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * vs_attn_aggregate_varlen -- vs_attn_aggregate for B sequences packed along
+ * the token axis (each sequence's weights are its own causal softmax; the
+ * sums are per sequence, at positions relative to its start).
+ *   total_tokens, cu_seqlens, max_seqlen  as for vs_sparse_attn_fwd_varlen
+ *            (cu_seqlens on the DEVICE; a malformed entry leaves that
+ *            sequence's entries of A_v unwritten and of A_s zero, and sets
+ *            VS_DEVFLAG_BOUNDS).
+ *   lse      fp32 [Hq][total_tokens] as written by vs_dense_attn_fwd_varlen.
+ *   A_v, A_s fp32 [Hq][total_tokens]: sequence b's column j at
+ *            h * total_tokens + cu_seqlens[b] + j, its offset o likewise.
+ */
+vs_status vs_attn_aggregate_varlen(const void* Q, const void* K, vs_dtype dtype, int total_tokens,
+                                   int B, const int32_t* cu_seqlens, int max_seqlen, int Hq,
+                                   int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                                   float softmax_scale, const float* lse, float* A_v, float* A_s,
+                                   void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Device status of the last call that used `ws`: synchronises `stream`,
  * copies the status word to `*flags` (VS_DEVFLAG_* bits) and returns VS_OK,
  * VS_ERR_DEVICE_TIMEOUT or VS_ERR_DEVICE_BOUNDS accordingly.

@@ -46,6 +46,7 @@ EXPORTS = (
     "vs_block_attn_workspace_size", "vs_block_sparse_attn_fwd", "vs_selftest_exp",
     "vs_block_select_workspace_size_varlen", "vs_block_select_varlen",
     "vs_block_attn_workspace_size_varlen", "vs_block_sparse_attn_fwd_varlen",
+    "vs_attn_aggregate_varlen",
 )
 
 
@@ -117,6 +118,9 @@ def lib() -> ctypes.CDLL:
         L.vs_block_sparse_attn_fwd_varlen.argtypes = [P, P, P, I, I, I, P, I, I, I, I, I64, I64, F,
                                                       P, P, P, P, Z, P]
         L.vs_block_sparse_attn_fwd_varlen.restype = I
+        L.vs_attn_aggregate_varlen.argtypes = [P, P, I, I, I, P, I, I, I, I, I64, I64, F, P, P,
+                                               P, P, Z, P]
+        L.vs_attn_aggregate_varlen.restype = I
         L.vs_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
         L.vs_read_device_status.restype = I
         L.vs_selftest_wait_timeout.argtypes = [P, U64, P]
@@ -262,6 +266,33 @@ def vs_dense_attn_fwd_varlen(Q, K, V, cu_seqlens, max_seqlen, O, lse, ws, softma
         _ptr(Q), _ptr(K), _ptr(V), _dtype(Q), T, B, _ptr(cu_seqlens), int(max_seqlen), Hq, Hkv, d,
         Q.stride(0), K.stride(0), float(softmax_scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
         _stream(stream)), "vs_dense_attn_fwd_varlen")
+
+
+def vs_attn_aggregate_varlen(Q, K, cu_seqlens, max_seqlen, lse, A_v, A_s, ws, softmax_scale=0.0,
+                             stream=None):
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    _check(lib().vs_attn_aggregate_varlen(
+        _ptr(Q), _ptr(K), _dtype(Q), T, B, _ptr(cu_seqlens), int(max_seqlen), Hq, Hkv, d,
+        Q.stride(0), K.stride(0), float(softmax_scale), _ptr(lse), _ptr(A_v), _ptr(A_s), _ptr(ws),
+        ws.numel(), _stream(stream)), "vs_attn_aggregate_varlen")
+
+
+def aggregate_varlen(Q, K, V, cu_seqlens, max_seqlen, ws=None, stream=None):
+    """Per-sequence column / diagonal sums of a packed batch, fp32 [Hq, total]
+    each: the batched dense forward for the row LSE, then the aggregation."""
+    T, Hq, _ = Q.shape
+    B = cu_seqlens.numel() - 1
+    ws = ws if ws is not None else workspace(256, Q.device)
+    O = torch.empty_like(Q)
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=Q.device)
+    wsd = workspace(vs_attn_workspace_size_varlen(B, max_seqlen, 1, Q.shape[2]), Q.device)
+    vs_dense_attn_fwd_varlen(Q, K, V, cu_seqlens, max_seqlen, O, lse, wsd, stream=stream)
+    A_v = torch.empty((Hq, T), dtype=torch.float32, device=Q.device)
+    A_s = torch.empty((Hq, T), dtype=torch.float32, device=Q.device)
+    vs_attn_aggregate_varlen(Q, K, cu_seqlens, max_seqlen, lse, A_v, A_s, ws, stream=stream)
+    return A_v, A_s
 
 
 def vs_block_select_workspace_size(N: int, Hkv: int, d: int) -> int:

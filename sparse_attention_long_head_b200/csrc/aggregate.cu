@@ -62,7 +62,10 @@ struct AggCfg {
 };
 
 struct AggParams {
-  int N, Hq, Hkv, G, T, num_units;
+  int N, Hq, Hkv, G, T, num_units;  // N, T: of the longest sequence
+  int B;                            // sequences
+  int64_t total;                    // token rows; lse, A_v, A_s are [Hq][total]
+  const int32_t* cu;                // sequence offsets (device) or null
   float scale_log2;
   const float* lse;
   float* Av;
@@ -71,20 +74,29 @@ struct AggParams {
   uint64_t wait_limit_ns;
 };
 
-// Unit u: heads in order, and within a head the longest walks (small b) first.
+// Unit u: sequences in order, then heads, and within a head the longest
+// walks (small b) first.  A key block past its sequence's end has n = 0 and
+// is skipped by every role.
 struct AggUnit {
   int h, b, n, n0, n1, st0, st1;
+  int seq, Nb;    // the unit's sequence and its tokens
+  int64_t tok0;   // its first token row
+  bool ok_seq;    // false: malformed offsets (the sequence is empty)
 };
 
 __device__ __forceinline__ AggUnit agg_unit(const AggParams& P, int u) {
   AggUnit a;
+  const int per_seq = P.Hq * P.T;
+  a.seq = u / per_seq;
+  u -= a.seq * per_seq;
+  a.ok_seq = seq_range(P.cu, P.total, P.N, a.seq, a.tok0, a.Nb);
   a.h = u / P.T;
   a.b = u - a.h * P.T;
-  a.n = P.T - a.b;
+  a.n = max(0, (a.Nb + 127) / 128 - a.b);
   a.n0 = (a.n + 1) / 2;
   a.n1 = a.n - a.n0;
   const uint32_t x = (uint32_t)a.b * 2654435761u + (uint32_t)a.h * 40503u;
-  a.st0 = (int)((x >> 8) % (uint32_t)a.n0);
+  a.st0 = a.n0 > 0 ? (int)((x >> 8) % (uint32_t)a.n0) : 0;
   a.st1 = a.n1 > 0 ? (int)((x >> 16) % (uint32_t)a.n1) : 0;
   return a;
 }
@@ -164,9 +176,10 @@ __global__ void __launch_bounds__(kAggThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
       const AggUnit a = agg_unit(P, u);
+      if (a.n == 0) continue;
       const int ng = grp == 0 ? a.n0 : a.n1;
-      const float* lse_h = P.lse + (int64_t)a.h * P.N;
-      float* As_h = P.As + (int64_t)a.h * P.N;
+      const float* lse_h = P.lse + (int64_t)a.h * P.total + a.tok0;
+      float* As_h = P.As + (int64_t)a.h * P.total + a.tok0;
       {
         uint32_t z[32];
 #pragma unroll
@@ -180,7 +193,7 @@ __global__ void __launch_bounds__(kAggThreads, 1)
       // this row's LSE for the walk's next tile, loaded a tile ahead
       auto lse_of = [&](int s) -> float {
         const int64_t ii = 128 * (int64_t)(a.b + agg_tile(a, grp, s)) + r;
-        return ii < P.N ? __ldg(lse_h + ii) : 0.f;
+        return ii < a.Nb ? __ldg(lse_h + ii) : 0.f;
       };
       float lse_next = ng > 0 ? lse_of(0) : 0.f;
       for (int s = 0; s < ng && ok; ++s, ++cnt) {
@@ -204,8 +217,9 @@ __global__ void __launch_bounds__(kAggThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(B_SEMPTY + grp));  // the S buffer may be overwritten
         const int64_t i = 128 * (int64_t)(a.b + j) + r;
-        // rows past N weigh nothing (their Q rows are zero-filled, so s is finite)
-        const float nl = i < P.N ? -lse_i * 1.4426950408889634f : -INFINITY;
+        // rows past the sequence's end weigh nothing (their Q rows are the next
+        // sequence's or zero-filled, so s is finite)
+        const float nl = i < a.Nb ? -lse_i * 1.4426950408889634f : -INFINITY;
         if (j == 0) {  // the diagonal tile: keys after the row weigh nothing
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -257,14 +271,14 @@ __global__ void __launch_bounds__(kAggThreads, 1)
         const int64_t oa = 128 * (int64_t)j - r;
         if (carry_off == oa) {
           da += carry;
-        } else if (carry_off >= 0 && carry_off < P.N && carry != 0.f) {
+        } else if (carry_off >= 0 && carry_off < a.Nb && carry != 0.f) {
           atomicAdd(As_h + carry_off, carry);
         }
-        if (oa >= 0 && oa < P.N && da != 0.f) atomicAdd(As_h + oa, da);
+        if (oa >= 0 && oa < a.Nb && da != 0.f) atomicAdd(As_h + oa, da);
         carry = db;
         carry_off = r > 0 ? oa + 128 : -1;
       }
-      if (ok && carry_off >= 0 && carry_off < P.N && carry != 0.f)
+      if (ok && carry_off >= 0 && carry_off < a.Nb && carry != 0.f)
         atomicAdd(As_h + carry_off, carry);
       // column sums of this group's accumulator through the skewed buffer
       float cs = 0.f;
@@ -294,7 +308,7 @@ __global__ void __launch_bounds__(kAggThreads, 1)
       }
       if (grp == 0) {
         const int64_t jcol = 128 * (int64_t)a.b + r;
-        if (jcol < P.N) P.Av[(int64_t)a.h * P.N + jcol] = cs + comb[r];
+        if (jcol < a.Nb) P.Av[(int64_t)a.h * P.total + a.tok0 + jcol] = cs + comb[r];
       }
       named_bar_sync(3, 256);  // comb is reused by the next unit
     }
@@ -308,6 +322,7 @@ __global__ void __launch_bounds__(kAggThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
         const AggUnit a = agg_unit(P, u);
+        if (a.n == 0) continue;
         if (!mbar_wait(bar(B_KFULL), kcount & 1, wc)) { ok = false; break; }
         // the halves alternate: group 0's step s, then group 1's step s
         for (int x = 0; x < a.n && ok; ++x, ++qseq) {
@@ -345,11 +360,14 @@ __global__ void __launch_bounds__(kAggThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < P.num_units && ok; u += gridDim.x) {
         const AggUnit a = agg_unit(P, u);
+        if (!a.ok_seq && a.h == 0 && a.b == 0) atomicOr(P.status, VS_DEVFLAG_BOUNDS);
+        if (a.n == 0) continue;
         const int g = a.h / P.G;
         if (kcount > 0 && !mbar_wait(bar(B_KEMPTY), (kcount - 1) & 1, wc)) { ok = false; break; }
         mbar_arrive_expect_tx(bar(B_KFULL), C::kTileBytes);
         for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_2d(smem_u32(sK + hh * 16384), &tmK, bar(B_KFULL), g * D + 64 * hh, 128 * a.b);
+          tma_load_2d(smem_u32(sK + hh * 16384), &tmK, bar(B_KFULL), g * D + 64 * hh,
+                      (int)(a.tok0 + 128 * a.b));
         ++kcount;
         for (int x = 0; x < a.n && ok; ++x, ++qseq) {
           const int s = x < 2 * a.n1 ? x >> 1 : x - a.n1;
@@ -364,7 +382,7 @@ __global__ void __launch_bounds__(kAggThreads, 1)
           mbar_arrive_expect_tx(bar(B_QFULL + qs), C::kTileBytes);
           for (int hh = 0; hh < D / 64; ++hh)
             tma_load_2d(smem_u32(sQ + qs * C::kTileBytes + hh * 16384), &tmQ, bar(B_QFULL + qs),
-                        a.h * D + 64 * hh, 128 * (a.b + j));
+                        a.h * D + 64 * hh, (int)(a.tok0 + 128 * (a.b + j)));
         }
       }
       // let every issued copy land before shared memory is released
@@ -389,8 +407,8 @@ cudaError_t launch_agg_impl(const AggArgs& a) {
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap mQ, mK;
   CUresult rc = CUDA_SUCCESS;
-  encode_rows_bf16_sw128(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.N, a.q_stride, &rc);
-  encode_rows_bf16_sw128(enc, &mK, a.K, (int64_t)a.Hkv * D, a.N, a.kv_stride, &rc);
+  encode_rows_bf16_sw128(enc, &mQ, a.Q, (int64_t)a.Hq * D, a.total, a.q_stride, &rc);
+  encode_rows_bf16_sw128(enc, &mK, a.K, (int64_t)a.Hkv * D, a.total, a.kv_stride, &rc);
   if (rc != CUDA_SUCCESS) return cudaErrorInvalidValue;
   AggParams P;
   P.N = a.N;
@@ -398,7 +416,10 @@ cudaError_t launch_agg_impl(const AggArgs& a) {
   P.Hkv = a.Hkv;
   P.G = a.Hq / a.Hkv;
   P.T = (a.N + 127) / 128;
-  P.num_units = a.Hq * P.T;
+  P.num_units = a.B * a.Hq * P.T;
+  P.B = a.B;
+  P.total = a.total;
+  P.cu = a.cu_seqlens;
   P.scale_log2 = a.scale * 1.4426950408889634f;
   P.lse = a.lse;
   P.Av = a.Av;

@@ -280,16 +280,19 @@ vs_status vs_dense_attn_fwd(const void* Q, const void* K, const void* V, vs_dtyp
                    ws_bytes, stream);
 }
 
-vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
-                            int d, int64_t q_stride_tok, int64_t kv_stride_tok,
-                            float softmax_scale, const float* lse, float* A_v, float* A_s,
-                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+static vs_status aggregate_impl(const void* Q, const void* K, vs_dtype dtype, int N, int B,
+                                int64_t total, const int32_t* cu, int Hq, int Hkv, int d,
+                                int64_t q_stride_tok, int64_t kv_stride_tok, float softmax_scale,
+                                const float* lse, float* A_v, float* A_s, void* ws,
+                                size_t ws_bytes, cudaStream_t stream) {
   if (!lse || !A_v || !A_s) return VS_ERR_INVALID_ARG;
   // the checks shared with attention (V and O stand in for K and A_v here)
   vs_status st = check_attn_common(Q, K, K, dtype, N, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
                                    softmax_scale, A_v);
   if (st != VS_OK) return st;
+  if (B < 1 || total < 1 || total > INT32_MAX) return VS_ERR_INVALID_ARG;
   if (dtype != VS_BF16) return VS_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hq * ((N + 127) / 128) >= ((int64_t)1 << 31)) return VS_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < kStatusBytes || !aligned(ws, 256)) return VS_ERR_WORKSPACE;
   AggArgs a;
   a.Q = Q;
@@ -298,6 +301,9 @@ vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N,
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.d = d;
+  a.B = B;
+  a.total = total;
+  a.cu_seqlens = cu;
   a.q_stride = q_stride_tok;
   a.kv_stride = kv_stride_tok;
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
@@ -307,9 +313,28 @@ vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N,
   a.status = static_cast<int*>(ws);
   a.stream = stream;
   if (cudaMemsetAsync(a.status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
-  if (cudaMemsetAsync(A_s, 0, sizeof(float) * (size_t)Hq * (size_t)N, stream) != cudaSuccess)
+  if (cudaMemsetAsync(A_s, 0, sizeof(float) * (size_t)Hq * (size_t)total, stream) != cudaSuccess)
     return VS_ERR_CUDA;
   return launch_aggregate(a) == cudaSuccess ? VS_OK : VS_ERR_CUDA;
+}
+
+vs_status vs_attn_aggregate(const void* Q, const void* K, vs_dtype dtype, int N, int Hq, int Hkv,
+                            int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                            float softmax_scale, const float* lse, float* A_v, float* A_s,
+                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return aggregate_impl(Q, K, dtype, N, 1, N, nullptr, Hq, Hkv, d, q_stride_tok, kv_stride_tok,
+                        softmax_scale, lse, A_v, A_s, ws, ws_bytes, stream);
+}
+
+vs_status vs_attn_aggregate_varlen(const void* Q, const void* K, vs_dtype dtype, int total_tokens,
+                                   int B, const int32_t* cu_seqlens, int max_seqlen, int Hq,
+                                   int Hkv, int d, int64_t q_stride_tok, int64_t kv_stride_tok,
+                                   float softmax_scale, const float* lse, float* A_v, float* A_s,
+                                   void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!cu_seqlens) return VS_ERR_INVALID_ARG;
+  return aggregate_impl(Q, K, dtype, max_seqlen, B, total_tokens, cu_seqlens, Hq, Hkv, d,
+                        q_stride_tok, kv_stride_tok, softmax_scale, lse, A_v, A_s, ws, ws_bytes,
+                        stream);
 }
 
 size_t vs_block_select_workspace_size(int N, int Hkv, int d) {

@@ -192,7 +192,10 @@ struct AttnArgs {
 struct AggArgs {
   const void* Q;
   const void* K;
-  int N, Hq, Hkv, d;
+  int N, Hq, Hkv, d;          // N: the longest sequence (the only one when B = 1)
+  int B;                      // sequences packed along the token axis
+  int64_t total;              // token rows of Q and K; lse, A_v, A_s are [Hq][total]
+  const int32_t* cu_seqlens;  // device [B + 1] or null
   int64_t q_stride, kv_stride;
   float scale;
   const float* lse;

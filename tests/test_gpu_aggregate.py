@@ -82,3 +82,32 @@ def test_full_size_tail_and_row_sums(name, cuda_device):
     for x, h in enumerate(heads):
         _check(A_v[h, N - R:], R_v[x, N - R:], f"{name} A_v tail head {h}")
         _check(A_s[h, N - R:], R_s[x, N - R:], f"{name} A_s tail head {h}")
+
+
+@pytest.mark.parametrize("lengths,d,Hq,Hkv", [((300, 1, 1000, 129, 2049), 128, 4, 2),
+                                              ((700, 256, 1500), 64, 2, 1)])
+def test_batched_sequences_against_oracle(lengths, d, Hq, Hkv, cuda_device):
+    # sequences packed along the token axis: each sequence's sums against the
+    # oracle on that sequence alone, and A_v equal bit for bit to the
+    # single-sequence call (A_v has no atomics)
+    parts = [gen_qkv(7 * n + b, n, Hq, Hkv, d, 10000.0) for b, n in enumerate(lengths)]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    Qc, Kc, Vc = (np.concatenate([p[t] for p in parts]) for t in range(3))
+    Q, K, V = bf16_to_dev(Qc), bf16_to_dev(Kc), bf16_to_dev(Vc)
+    ws = vs.workspace(256)
+    A_v, A_s = vs.aggregate_varlen(Q, K, V, torch.from_numpy(cu).cuda(), max(lengths), ws=ws)
+    torch.cuda.synchronize()
+    rc, flags = vs.vs_read_device_status(ws)
+    assert rc == vs.VS_OK and flags == 0
+    Av = A_v.cpu().numpy().astype(np.float64)
+    As = A_s.cpu().numpy().astype(np.float64)
+    for b, (Qb, Kb, Vb) in enumerate(parts):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        n = t1 - t0
+        R_v, R_s = oracle.aggregate(Qb, Kb)
+        _check(Av[:, t0:t1], R_v, f"seq {b} A_v")
+        _check(As[:, t0:t1], R_s, f"seq {b} A_s")
+        assert np.allclose(Av[:, t0:t1].sum(1), n, rtol=1e-4)
+        assert np.allclose(As[:, t0:t1].sum(1), n, rtol=1e-4)
+        S_v, _ = _gpu_aggregate(Qb, Kb, Vb)
+        assert np.array_equal(S_v, Av[:, t0:t1]), b
