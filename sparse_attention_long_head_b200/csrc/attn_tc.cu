@@ -533,43 +533,12 @@ __device__ __forceinline__ bool item_mask(const AttnParams& P, const UnitInfo& u
   return true;
 }
 
-// 2^x on the FMA pipe for a pair of lanes: k = round(x) via the 1.5 * 2^23
-// shifter, f = x - k in [-1/2, 1/2], 2^f by a degree-3 polynomial
-// (coefficients from csrc/fit_exp2_poly.py, max relative error 7.5e-5), and
-// 2^k added to the exponent field.  x is clamped to >= -125 so the exponent
-// stays normal; callers zero masked lanes themselves.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f,
-                  kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-// Which column pairs of a 128-column row take the FMA-pipe exp2 (the rest use
-// MUFU.EX2): kPolyNum out of every kPolyDen pairs.
-#ifndef VS_POLY_NUM
-#define VS_POLY_NUM 0
-#endif
-#ifndef VS_POLY_DEN
-#define VS_POLY_DEN 8
-#endif
-__host__ __device__ constexpr bool poly_pair(int j) { return (j % VS_POLY_DEN) < VS_POLY_NUM; }
-
 // p = 2^(s * scale_log2 - m) for one 128-column row (s is already -inf where
 // masked), packed to bf16 pairs and stored over the row's S columns in TMEM
 // 32 columns at a time (all of S is already in registers), row sum into ls.
 // One call site only: two inlined copies make the compiler spill the row.
-__device__ __forceinline__ void exp_tile(const uint32_t (&sr)[4][32], const uint32_t (&mw)[4],
-                                         bool masked, float sl2, float m_base, uint32_t tS,
-                                         float& ls) {
+__device__ __forceinline__ void exp_tile(const uint32_t (&sr)[4][32], float sl2, float m_base,
+                                         uint32_t tS, float& ls) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -578,19 +547,8 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&sr)[4][32], const uint
     for (int c = 0; c < 32; c += 2) {
       const float x0 = fmaf(__uint_as_float(sr[q][c]), sl2, -m_base);
       const float x1 = fmaf(__uint_as_float(sr[q][c + 1]), sl2, -m_base);
-      float p0, p1;
-      if (poly_pair(q * 16 + c / 2)) {
-        const float2 pp = exp2_fma2(make_float2(x0, x1));
-        p0 = pp.x;
-        p1 = pp.y;
-        if (masked) {
-          if (!((mw[q] >> c) & 1u)) p0 = 0.f;
-          if (!((mw[q] >> (c + 1)) & 1u)) p1 = 0.f;
-        }
-      } else {
-        p0 = ex2_approx(x0);
-        p1 = ex2_approx(x1);
-      }
+      const float p0 = ex2_approx(x0);
+      const float p1 = ex2_approx(x1);
       acc[(c >> 1) & 1] += p0;
       acc[2 + ((c >> 1) & 1)] += p1;
       pk[c / 2] = pack_bf16x2(p0, p1);
@@ -745,7 +703,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         const float m_base = m_use == -INFINITY ? 0.f : m_use;
         float ls = 0.f;
-        exp_tile(sr, mw, masked, P.scale_log2, m_base, tS, ls);
+        exp_tile(sr, P.scale_log2, m_base, tS, ls);
         l += ls;
         if (nproc > 0 && __any_sync(0xffffffffu, need)) {
           // O must be rescaled before PV(k) accumulates into it; the previous
