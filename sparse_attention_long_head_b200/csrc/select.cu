@@ -20,12 +20,16 @@
 //   * The threshold rule keeps k = min(k_threshold, cap) entries, so its mass
 //     matters only when the top-cap entries already reach tau * Z.  The kernel
 //     takes Z in one pass (fixed-order fp64 sum), runs the count search for
-//     the cap, and sums the top-cap entries' mass; only when that reaches
-//     tau * Z does the mass search run, and then over the keys at or above
-//     the cap's boundary key alone (packed in index order into a short list
-//     when it fits): every key of the threshold's prefix is among them.  A
+//     the cap, packs the keys at or above the cap's boundary key in index
+//     order into a short list (when it fits) and sums the top-cap entries'
+//     mass from it; only when that reaches tau * Z does the mass search run,
+//     over the same list: every key of the threshold's prefix is in it.  A
 //     key's mass is exp(s - s_max) in fp64 (Tang's table-driven method,
 //     exp64.cuh).
+//   * Each pass's decision is taken by one warp: lane l holds eight buckets
+//     of the merged histogram, a shuffle scan of the lanes' sums (counts, or
+//     fp64 masses) finds the lane where the target is reached, and that lane
+//     walks its eight buckets.
 //   * The mass histogram takes no fp64 atomics (shared-memory fp64 atomic
 //     adds cost more than half of this kernel's time when they were used,
 //     by measurement): each warp owns a private copy; lanes holding
@@ -407,30 +411,72 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
           sh.cabove_c = ca;
         }
       }
-      if (do_mass && tid == 32) {  // mass path: first bucket reaching the target
-        int bs = -1, last_nonempty = -1;
-        uint32_t ca = cab_t;
-        double ma = mab_t;
-        for (int b = 255; b >= 0; --b) {
-          const uint32_t c = sh.tot_ct[b];
-          if (c == 0) continue;
-          last_nonempty = b;
-          if (ma + sh.tot_mt[b] >= target) {
-            bs = b;
-            break;
+      if (do_mass && tid >= 32 && tid < 64) {
+        // mass path: the first bucket from the top at which the running mass
+        // reaches the target.  Lane l holds buckets 255 - 8 l .. 248 - 8 l;
+        // an inclusive scan of the lanes' sums finds the lane, which walks its
+        // eight buckets.  (Fixed order, the same in every CTA of the cluster.)
+        const int lane = tid - 32;
+        uint32_t c[8], csum = 0;
+        double m[8], msum = 0.0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          c[j] = sh.tot_ct[255 - 8 * lane - j];
+          m[j] = sh.tot_mt[255 - 8 * lane - j];
+          csum += c[j];
+          msum += m[j];
+        }
+        uint32_t cincl = csum;
+        double mincl = msum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t yc = __shfl_up_sync(0xffffffffu, cincl, o);
+          const double ym = __shfl_up_sync(0xffffffffu, mincl, o);
+          if (lane >= o) {
+            cincl += yc;
+            mincl += ym;
           }
-          ca += c;
-          ma += sh.tot_mt[b];
         }
-        if (bs < 0) {  // rounding left the total just short: take the last group
-          bs = last_nonempty;
-          ca -= sh.tot_ct[bs];
-          ma -= sh.tot_mt[bs];
+        uint32_t cex = __shfl_up_sync(0xffffffffu, cincl, 1);
+        double mex = __shfl_up_sync(0xffffffffu, mincl, 1);
+        if (lane == 0) {
+          cex = 0;
+          mex = 0.0;
         }
-        sh.bstar_t = bs;
-        sh.cabove_t = ca;
-        sh.mabove_t = ma;
-        sh.eqcnt_t = sh.tot_ct[bs];
+        const unsigned hit = __ballot_sync(0xffffffffu, mab_t + mincl >= target);
+        // no lane reaches it (rounding left the total just short): the last
+        // non-empty bucket is the group, with every other bucket above it
+        const unsigned nonempty = __ballot_sync(0xffffffffu, csum != 0);
+        const int wl = hit ? __ffs(hit) - 1 : (nonempty ? 31 - __clz(nonempty) : 0);
+        if (lane == wl) {
+          int bs = -1, last_j = -1;
+          uint32_t ca = cab_t + cex;
+          double ma = mab_t + mex;
+          uint32_t ca_last = ca;
+          double ma_last = ma;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (bs >= 0 || c[j] == 0) continue;
+            if (hit && ma + m[j] >= target) {
+              bs = 255 - 8 * lane - j;
+            } else {
+              last_j = j;
+              ca_last = ca;
+              ma_last = ma;
+              ca += c[j];
+              ma += m[j];
+            }
+          }
+          if (bs < 0) {  // the lane's last non-empty bucket
+            bs = last_j >= 0 ? 255 - 8 * lane - last_j : 0;
+            ca = ca_last;
+            ma = ma_last;
+          }
+          sh.bstar_t = bs;
+          sh.cabove_t = ca;
+          sh.mabove_t = ma;
+          sh.eqcnt_t = sh.tot_ct[bs];
+        }
       }
       __syncthreads();
       if (do_count) {
@@ -457,12 +503,52 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
     cabove = static_cast<uint32_t>(k_count);
   }
   if (thr) {
+    // The keys at or above the cap's boundary key (scattered over the row)
+    // are packed in index order into a short list when it fits: the top-cap
+    // mass and, when it reaches tau * Z, the mass search read only them.
+    {
+      const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+      const int wper = ((n + nw - 1) / nw + 31) / 32 * 32;
+      const int wb = min(n, warp * wper), wend = min(n, wb + wper);
+      uint32_t c = 0;
+      for (int base = wb; base < wend; base += 32) {
+        const int e = base + lane;
+        c += __popc(__ballot_sync(0xffffffffu, e < wend && key_at(e) >= pf_c));
+      }
+      if (lane == 0) sh.wg[warp] = c;
+      __syncthreads();
+      int off = 0;
+      for (int w = 0; w < nw; ++w) {
+        if (w < warp) off += static_cast<int>(sh.wg[w]);
+        ncand += static_cast<int>(sh.wg[w]);
+      }
+      use_list = ncand <= a.list_cap;
+      if (use_list) {
+        const unsigned lt = (1u << lane) - 1u;
+        for (int base = wb; base < wend; base += 32) {
+          const int e = base + lane;
+          const uint32_t k = e < wend ? key_at(e) : 0u;
+          const bool in = e < wend && k >= pf_c;
+          const unsigned m = __ballot_sync(0xffffffffu, in);
+          if (in) clist[off + __popc(m & lt)] = k;
+          off += __popc(m);
+        }
+      }
+      __syncthreads();
+    }
     // mass of the top-cap entries: the keys above the cap's boundary key,
     // and as many copies of that key's mass as the cap keeps
     double mp = 0.0;
-    for (int e = tid; e < n; e += nt) {
-      const uint32_t k = key_at(e);
-      if (k > pf_c) mp += pmass(k, kmax, smax, tab);
+    if (use_list) {
+      for (int e = tid; e < ncand; e += nt) {
+        const uint32_t k = clist[e];
+        if (k > pf_c) mp += pmass(k, kmax, smax, tab);
+      }
+    } else {
+      for (int e = tid; e < n; e += nt) {
+        const uint32_t k = key_at(e);
+        if (k > pf_c) mp += pmass(k, kmax, smax, tab);
+      }
     }
     mp = block_reduce<double>(mp, sh.wred_d, [](double x, double y) { return x + y; });
     if (tid == 0) sh.mpart = mp;
@@ -471,40 +557,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
     for (int r = 0; r < C; ++r) mcap += *cl.map_shared_rank(&sh.mpart, r);
     mcap += static_cast<double>(k_count - static_cast<int>(cab_c)) * pmass(pf_c, kmax, smax, tab);
     if (mcap >= target) {
-      // The threshold's prefix ends within the top-cap entries.  Their keys
-      // (>= the cap's boundary key; scattered over the row) are first packed
-      // in index order into a short list when it fits, so the four passes
-      // read only them.
-      {
-        const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
-        const int wper = ((n + nw - 1) / nw + 31) / 32 * 32;
-        const int wb = min(n, warp * wper), wend = min(n, wb + wper);
-        uint32_t c = 0;
-        for (int base = wb; base < wend; base += 32) {
-          const int e = base + lane;
-          c += __popc(__ballot_sync(0xffffffffu, e < wend && key_at(e) >= pf_c));
-        }
-        if (lane == 0) sh.wg[warp] = c;
-        __syncthreads();
-        int off = 0;
-        for (int w = 0; w < nw; ++w) {
-          if (w < warp) off += static_cast<int>(sh.wg[w]);
-          ncand += static_cast<int>(sh.wg[w]);
-        }
-        use_list = ncand <= a.list_cap;
-        if (use_list) {
-          const unsigned lt = (1u << lane) - 1u;
-          for (int base = wb; base < wend; base += 32) {
-            const int e = base + lane;
-            const uint32_t k = e < wend ? key_at(e) : 0u;
-            const bool in = e < wend && k >= pf_c;
-            const unsigned m = __ballot_sync(0xffffffffu, in);
-            if (in) clist[off + __popc(m & lt)] = k;
-            off += __popc(m);
-          }
-        }
-        __syncthreads();
-      }
+      // the threshold's prefix ends within the top-cap entries
       radix(false, true, pf_c);
       // within the final group of equal keys every entry has the same mass
       const double pstar = pmass(pf_t, kmax, smax, tab);
