@@ -156,6 +156,17 @@ def copy_heads(dst, src, h0, h1, stream):
         raise RuntimeError(f"cudaMemcpy2DAsync failed ({rc})")
 
 
+def copy_columns(dst, src, c0, c1, stream):
+    """Copy columns [c0, c1) of a row-major [R, C] tensor from pinned host
+    memory to the device, as one strided copy on `stream`."""
+    R, C = src.shape
+    es = src.element_size()
+    rc = _cudart().cudaMemcpy2DAsync(dst.data_ptr() + c0 * es, C * es, src.data_ptr() + c0 * es,
+                                     C * es, (c1 - c0) * es, R, 1, stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"cudaMemcpy2DAsync failed ({rc})")
+
+
 def e2e_units(Hkv: int, G: int, head_cost, in_head_ms: float, kv_ms: float, out_head_ms: float,
               launch_ms: float = 0.05):
     """Order of the end-to-end pipeline's units: [(kv_group, h0, h1)].
@@ -962,15 +973,17 @@ def run_batch(args, w):
     cu = torch.from_numpy(cu_h).to(dev)
     max_n = int(max(w.lengths))
     cap_max = w.cap(max_n)
-    LV = [torch.from_numpy(lv).to(dev) for lv, _ in scores]
-    LS = [torch.from_numpy(ls).to(dev) for _, ls in scores]
+    # scores packed along the token axis: [H_sel][total], sequence b at cu[b]
+    LV = torch.from_numpy(np.ascontiguousarray(np.concatenate([lv for lv, _ in scores], 1))).to(dev)
+    LS = torch.from_numpy(np.ascontiguousarray(np.concatenate([ls for _, ls in scores], 1))).to(dev)
+    caps = torch.tensor([w.cap(n) for n in w.lengths], dtype=torch.int32, device=dev)
     vi = torch.full((B * H_sel, cap_max), -1, dtype=torch.int32, device=dev)
     si = torch.full_like(vi, -1)
     vc = torch.empty(B * H_sel, dtype=torch.int32, device=dev)
     sc = torch.empty_like(vc)
     O = torch.empty_like(Q)
     lse = torch.empty((Hq, T), dtype=torch.float32, device=dev)
-    ws_sel = [vs.workspace(vs.vs_select_workspace_size(H_sel, n), dev) for n in w.lengths]
+    ws_sel = vs.workspace(vs.vs_select_workspace_size_varlen(B, H_sel, max_n), dev)
     ws_att = vs.workspace(vs.vs_attn_workspace_size_varlen(B, max_n, H_sel, d, cap_max), dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     ev = {k: [] for k in ("s0", "a0", "a1")}
@@ -980,11 +993,8 @@ def run_batch(args, w):
             e = torch.cuda.Event(enable_timing=True)
             e.record(stream)
             ev["s0"].append(e)
-        for b, n in enumerate(w.lengths):
-            rows = slice(b * H_sel, (b + 1) * H_sel)
-            k = w.cap(n)
-            vs.vs_select(LV[b], mode, k, w.tau_v, vi[rows], vc[rows], ws_sel[b])
-            vs.vs_select(LS[b], mode, k, w.tau_s, si[rows], sc[rows], ws_sel[b])
+        vs.vs_select_varlen(LV, cu, max_n, mode, caps, cap_max, w.tau_v, vi, vc, ws_sel)
+        vs.vs_select_varlen(LS, cu, max_n, mode, caps, cap_max, w.tau_s, si, sc, ws_sel)
         if record:
             e = torch.cuda.Event(enable_timing=True)
             e.record(stream)
@@ -1052,9 +1062,9 @@ def run_batch(args, w):
     if not args.no_e2e:
         hQ, hK, hV = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
                       for x in (Qb, Kb, Vb))
-        hS = [torch.from_numpy(x).pin_memory() for pair in scores for x in pair]
+        hLV, hLS = LV.cpu().pin_memory(), LS.cpu().pin_memory()  # packed [H_sel][total]
         hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in [hQ, hK, hV] + hS)
+        h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hLV, hLS))
         d2h = hO.numel() * hO.element_size()
         bounds, acc = [0], 0
         for b, n in enumerate(w.lengths):
@@ -1070,6 +1080,7 @@ def run_batch(args, w):
                  for b0, b1 in chunks]
         maxn_c = [int(max(w.lengths[b0:b1])) for b0, b1 in chunks]
         ws_att2 = [ws_att, vs.workspace(ws_att.numel(), dev)]
+        ws_sel2 = [ws_sel, vs.workspace(ws_sel.numel(), dev)]
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         cs = [stream, torch.cuda.Stream(dev)]
 
@@ -1085,9 +1096,8 @@ def run_batch(args, w):
                     Q[t0:t1].copy_(hQ[t0:t1], non_blocking=True)
                     K[t0:t1].copy_(hK[t0:t1], non_blocking=True)
                     V[t0:t1].copy_(hV[t0:t1], non_blocking=True)
-                    for b in range(b0, b1):
-                        LV[b].copy_(hS[2 * b], non_blocking=True)
-                        LS[b].copy_(hS[2 * b + 1], non_blocking=True)
+                    copy_columns(LV, hLV, t0, t1, s_in)
+                    copy_columns(LS, hLS, t0, t1, s_in)
                 e = torch.cuda.Event()
                 e.record(s_in)
                 landed.append(e)
@@ -1098,13 +1108,12 @@ def run_batch(args, w):
                 t0, t1 = int(cu_h[b0]), int(cu_h[b1])
                 r0, r1 = b0 * H_sel, b1 * H_sel
                 with torch.cuda.stream(st):
-                    for b in range(b0, b1):
-                        rows = slice(b * H_sel, (b + 1) * H_sel)
-                        k = w.cap(w.lengths[b])
-                        vs.vs_select(LV[b], mode, k, w.tau_v, vi[rows], vc[rows], ws_sel[b],
-                                     stream=st)
-                        vs.vs_select(LS[b], mode, k, w.tau_s, si[rows], sc[rows], ws_sel[b],
-                                     stream=st)
+                    # the chunk's sequences: their offsets into the packed scores
+                    cu_j, caps_j = cu[b0:b1 + 1], caps[b0:b1]
+                    vs.vs_select_varlen(LV, cu_j, maxn_c[j], mode, caps_j, cap_max, w.tau_v,
+                                        vi[r0:r1], vc[r0:r1], ws_sel2[j % 2], stream=st)
+                    vs.vs_select_varlen(LS, cu_j, maxn_c[j], mode, caps_j, cap_max, w.tau_s,
+                                        si[r0:r1], sc[r0:r1], ws_sel2[j % 2], stream=st)
                     vs.vs_sparse_attn_fwd_varlen(Q[t0:t1], K[t0:t1], V[t0:t1], cu_c[j], maxn_c[j],
                                                  vi[r0:r1], vc[r0:r1], si[r0:r1], sc[r0:r1],
                                                  O[t0:t1], lse_c[j], ws_att2[j % 2], stream=st)
@@ -1135,8 +1144,8 @@ def run_batch(args, w):
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "protocol": E2E_PROTOCOL,
                "pipeline": f"{len(chunks)} chunks of consecutive sequences: copy-in stream, two "
-                           "alternating compute streams (selects + one batched attention call per "
-                           "chunk), copy-out stream"}
+                           "alternating compute streams (two batched selects + one batched "
+                           "attention call per chunk), copy-out stream"}
     peaks, peak_kind = measured_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     algo_bytes = (Q.numel() + K.numel() + V.numel() + O.numel()) * 2 + lse.numel() * 4 \

@@ -146,6 +146,38 @@ vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_sel
                     void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * vs_select_varlen -- vs_select for B sequences packed along the token axis,
+ * in one launch (the budget step of a batched prefill: each sequence's
+ * vertical or slash scores select that sequence's index set).
+ *   scores     fp32 [H][total_tokens] (device): head h of sequence b is
+ *              scores[h * total_tokens + cu_seqlens[b] + j], j < n_b.
+ *   cu_seqlens int32 [B + 1] (device), as for vs_sparse_attn_fwd_varlen;
+ *              max_seqlen >= every n_b (host; sizes the launch).
+ *   caps       int32 [B] (device): k_or_cap of sequence b, 1 <= caps[b] <=
+ *              n_b and <= cap_max; cap_max >= 1 and ld_idx >= cap_max.
+ *   mode, tau  as for vs_select, applied to every row.
+ *   idx        int32 [B * H][ld_idx] (device): row b * H + h as vs_select's
+ *              row for that sequence and head (indices from the sequence's
+ *              start, ascending, then -1 up to caps[b]; entries past caps[b]
+ *              untouched) -- the layout vs_sparse_attn_fwd_varlen reads.
+ *   count      int32 [B * H] (device).
+ *   ws         device workspace of at least
+ *              vs_select_workspace_size_varlen(B, H, max_seqlen) bytes,
+ *              256-byte aligned (status word).
+ * A sequence with n_b = 0 keeps nothing (count 0, its rows untouched).  A
+ * malformed offset or cap empties that sequence the same way and sets
+ * VS_DEVFLAG_BOUNDS.  B * H <= 65535; max_seqlen <= 2^20.  The fp64 sums
+ * are in a fixed order for a given (B, H, max_seqlen) and device, as for
+ * vs_select (the order follows the cluster the launcher picks for B * H rows
+ * of max_seqlen, so it may differ from a single-sequence call's).
+ */
+size_t vs_select_workspace_size_varlen(int B, int H, int max_seqlen);
+vs_status vs_select_varlen(const float* scores, int total_tokens, int B, const int32_t* cu_seqlens,
+                           int max_seqlen, int H, vs_select_mode mode, const int32_t* caps,
+                           int cap_max, double tau, int32_t* idx, int64_t ld_idx, int32_t* count,
+                           void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * vs_sparse_attn_fwd -- causal vertical-slash sparse attention forward
  * (Technical Summary, section 2, "Fused Kernel Execution": the vertical and
  * slash index lists are merged on the fly inside a FlashAttention-style

@@ -46,7 +46,7 @@ EXPORTS = (
     "vs_block_attn_workspace_size", "vs_block_sparse_attn_fwd", "vs_selftest_exp",
     "vs_block_select_workspace_size_varlen", "vs_block_select_varlen",
     "vs_block_attn_workspace_size_varlen", "vs_block_sparse_attn_fwd_varlen",
-    "vs_attn_aggregate_varlen",
+    "vs_attn_aggregate_varlen", "vs_select_workspace_size_varlen", "vs_select_varlen",
 )
 
 
@@ -80,6 +80,10 @@ def lib() -> ctypes.CDLL:
         L.vs_select_workspace_size.restype = Z
         L.vs_select.argtypes = [P, I, I, I64, I, I, D, P, I64, P, P, Z, P]
         L.vs_select.restype = I
+        L.vs_select_workspace_size_varlen.argtypes = [I, I, I]
+        L.vs_select_workspace_size_varlen.restype = Z
+        L.vs_select_varlen.argtypes = [P, I, I, P, I, I, I, P, I, D, P, I64, P, P, Z, P]
+        L.vs_select_varlen.restype = I
         L.vs_attn_workspace_size.argtypes = [I, I, I, I]
         L.vs_attn_workspace_size.restype = Z
         L.vs_attn_workspace_size_ld.argtypes = [I, I, I, I, I64]
@@ -199,6 +203,24 @@ def vs_select(scores, mode, k_or_cap, tau, idx, count, ws, stream=None):
     _check(lib().vs_select(_ptr(scores), H, N, scores.stride(0), int(mode), int(k_or_cap),
                            float(tau), _ptr(idx), idx.stride(0), _ptr(count), _ptr(ws), ws.numel(),
                            _stream(stream)), "vs_select")
+
+
+def vs_select_workspace_size_varlen(B: int, H: int, max_seqlen: int) -> int:
+    return lib().vs_select_workspace_size_varlen(B, H, max_seqlen)
+
+
+def vs_select_varlen(scores, cu_seqlens, max_seqlen, mode, caps, cap_max, tau, idx, count, ws,
+                     stream=None):
+    """scores fp32 [H, total_tokens] (contiguous rows); cu_seqlens int32 [B + 1] and caps int32
+    [B] on the device; idx int32 [B * H, ld_idx >= cap_max]; count int32 [B * H]; ws from
+    vs_select_workspace_size_varlen."""
+    H, total = scores.shape
+    B = cu_seqlens.numel() - 1
+    assert scores.stride(1) == 1 and scores.stride(0) == total
+    _check(lib().vs_select_varlen(_ptr(scores), total, B, _ptr(cu_seqlens), int(max_seqlen), H,
+                                  int(mode), _ptr(caps), int(cap_max), float(tau), _ptr(idx),
+                                  idx.stride(0), _ptr(count), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "vs_select_varlen")
 
 
 def vs_sparse_attn_fwd(Q, K, V, v_idx, v_cnt, s_idx, s_cnt, O, lse, ws, softmax_scale=0.0,
@@ -413,6 +435,20 @@ def select(scores, mode, k_or_cap, tau=1.0, ws=None, stream=None):
     cnt = torch.empty(H, dtype=torch.int32, device=scores.device)
     ws = workspace(vs_select_workspace_size(H, N), scores.device) if ws is None else ws
     vs_select(scores, mode, k_or_cap, tau, idx, cnt, ws, stream)
+    return idx, cnt
+
+
+def select_varlen(scores, cu_seqlens, max_seqlen, mode, caps, cap_max, tau=1.0, ws=None,
+                  stream=None):
+    """Allocates outputs and runs vs_select_varlen -> (idx [B * H, cap_max] filled with -1 past
+    each row's cap, count [B * H])."""
+    H = scores.shape[0]
+    B = cu_seqlens.numel() - 1
+    idx = torch.full((B * H, cap_max), -1, dtype=torch.int32, device=scores.device)
+    cnt = torch.empty(B * H, dtype=torch.int32, device=scores.device)
+    if ws is None:
+        ws = workspace(vs_select_workspace_size_varlen(B, H, max_seqlen), scores.device)
+    vs_select_varlen(scores, cu_seqlens, max_seqlen, mode, caps, cap_max, tau, idx, cnt, ws, stream)
     return idx, cnt
 
 

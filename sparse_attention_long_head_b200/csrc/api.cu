@@ -144,6 +144,36 @@ vs_status vs_select(const float* scores, int H, int N, int64_t ld_scores, vs_sel
   return VS_OK;
 }
 
+size_t vs_select_workspace_size_varlen(int B, int H, int max_seqlen) {
+  (void)B;
+  (void)H;
+  (void)max_seqlen;
+  return kStatusBytes;
+}
+
+vs_status vs_select_varlen(const float* scores, int total_tokens, int B, const int32_t* cu_seqlens,
+                           int max_seqlen, int H, vs_select_mode mode, const int32_t* caps,
+                           int cap_max, double tau, int32_t* idx, int64_t ld_idx, int32_t* count,
+                           void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!scores || !cu_seqlens || !caps || !idx || !count) return VS_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || (int64_t)B * H > 65535 || max_seqlen < 1 || total_tokens < 1)
+    return VS_ERR_INVALID_ARG;
+  if (max_seqlen > (1 << 20)) return VS_ERR_UNSUPPORTED;
+  if (mode != VS_SELECT_TOPK && mode != VS_SELECT_THRESHOLD && mode != VS_SELECT_MAXFRAC)
+    return VS_ERR_INVALID_ARG;
+  if (cap_max < 1 || ld_idx < cap_max) return VS_ERR_INVALID_ARG;
+  if (mode != VS_SELECT_TOPK && !(tau > 0.0 && tau <= 1.0)) return VS_ERR_INVALID_ARG;
+  const double ln_alpha = mode == VS_SELECT_MAXFRAC ? std::log(tau) : 0.0;
+  if (!ws || ws_bytes < vs_select_workspace_size_varlen(B, H, max_seqlen) || !aligned(ws, 256))
+    return VS_ERR_WORKSPACE;
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return VS_ERR_CUDA;
+  if (launch_select(scores, H, max_seqlen, total_tokens, mode, cap_max, tau, ln_alpha, idx, ld_idx,
+                    count, status, stream, cu_seqlens, total_tokens, caps, B) != cudaSuccess)
+    return VS_ERR_CUDA;
+  return VS_OK;
+}
+
 size_t vs_attn_workspace_size_ld(int N, int Hq, int H_sel, int d, int64_t v_ld) {
   (void)Hq;
   if (N < 1 || H_sel < 1 || (d != 64 && d != 128) || v_ld < 1) return kStatusBytes;

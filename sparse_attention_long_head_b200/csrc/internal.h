@@ -230,9 +230,12 @@ cudaError_t launch_pack(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_block_plan(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, const PlanLayout& L);
 cudaError_t launch_attn_fp32(const AttnArgs& a, const PlanLayout& L);
+// Batched form: cu (device, B + 1 offsets) and caps (device, B) non-null, N
+// the longest sequence, k_or_cap the bound on the caps, scores [H][total].
 cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,
                           double tau, double ln_alpha, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
-                          cudaStream_t stream);
+                          cudaStream_t stream, const int32_t* cu = nullptr, int64_t total = 0,
+                          const int32_t* caps = nullptr, int B = 1);
 cudaError_t launch_index_scores(const void* K, const void* V, int dtype, int N, int Hkv, int d,
                                 int64_t stride_tok, int64_t stride_head, const float* W1,
                                 const float* W2, int hidden, float* lv, float* ls,

@@ -86,6 +86,13 @@ struct SelArgs {
   int* status;
   int chunk;
   int list_cap;  // threshold rule: room for the mass search's candidate keys (after wmass)
+  // Batch of sequences (null cu: one score row per head).  Row b * H + h of
+  // the grid is sequence b of head h: scores at h * total + cu[b], its cap
+  // caps[b] (N: the longest sequence; k_or_cap: the bound on the caps).
+  const int32_t* cu;
+  int64_t total;
+  const int32_t* caps;
+  int H;
 };
 
 struct SelShared {
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   cg::cluster_group cl = cg::this_cluster();
   const int rank = static_cast<int>(cl.block_rank());
   const int C = static_cast<int>(cl.num_blocks());
-  const int h = blockIdx.y;
+  const int row_id = blockIdx.y;
   const int tid = threadIdx.x, nt = blockDim.x;
   extern __shared__ uint32_t skeys[];
   __shared__ SelShared sh;
@@ -171,9 +178,30 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   int ncand = 0;          // candidate keys of this CTA
   bool use_list = false;  // the mass search reads clist (else every key, filtered)
 
-  const float* row = a.scores + (int64_t)h * a.ld;
-  const int lo = rank * a.chunk;
-  const int n = max(0, min(a.N, lo + a.chunk) - lo);
+  const float* row = a.scores + (int64_t)row_id * a.ld;
+  int N = a.N, chunk = a.chunk, kcap = a.k_or_cap;
+  if (a.cu) {
+    // One row of a batch; every CTA of the cluster reads the same row, so
+    // they all leave here together when it keeps nothing.
+    const int b = row_id / a.H, hh = row_id - b * a.H;
+    int64_t t0;
+    int nb;
+    const bool ok_seq = seq_range(a.cu, a.total, a.N, b, t0, nb);
+    const int cap = ok_seq && nb > 0 ? __ldg(a.caps + b) : 0;
+    const bool ok_cap = nb == 0 || (cap >= 1 && cap <= nb && cap <= a.k_or_cap);
+    if ((!ok_seq || !ok_cap) && rank == 0 && tid == 0 && hh == 0)
+      atomicOr(a.status, VS_DEVFLAG_BOUNDS);
+    if (!ok_seq || !ok_cap || nb == 0) {  // an empty or malformed sequence keeps nothing
+      if (rank == 0 && tid == 0) a.count[row_id] = 0;
+      return;
+    }
+    N = nb;
+    chunk = (nb + C - 1) / C;
+    kcap = cap;
+    row = a.scores + (int64_t)hh * a.total + t0;
+  }
+  const int lo = rank * chunk;
+  const int n = max(0, min(N, lo + chunk) - lo);
   auto key_at = [&](int e) -> uint32_t { return CACHE ? skeys[e] : fkey(__ldg(row + lo + e)); };
 
   if (tid < 32) sh.exp_tab[tid] = exp2((double)tid / 32.0);  // read after the cluster barrier below
@@ -201,7 +229,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
   //     of the top-cap entries; only when that reaches tau * Z does the mass
   //     search run, and only over the keys at or above the cap's boundary key
   //     (every key of the threshold's prefix is among them).
-  int k_count = a.k_or_cap;
+  int k_count = kcap;
   bool thr = false;              // threshold rule with tau < 1 and a non-NaN maximum
   bool search = true;            // false: the kept set is every key >= kmin_kept
   uint32_t kmin_kept = 0xFFFFFFFFu;
@@ -236,7 +264,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
     }
     if (kmax == 0u) {  // every score is NaN: keep one entry
       k_count = 1;
-    } else if (tot <= a.k_or_cap) {
+    } else if (tot <= kcap) {
       k_count = tot;
       search = false;
     }
@@ -252,7 +280,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
       cl.sync();
       int tot = 0;
       for (int r = 0; r < C; ++r) tot += static_cast<int>(*cl.map_shared_rank(&sh.npos, r));
-      k_count = min(max(tot, 1), a.k_or_cap);
+      k_count = min(max(tot, 1), kcap);
     } else {
       thr = true;
     }
@@ -564,7 +592,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
       double mm = pstar > 0.0 ? ceil((target - mab_t) / pstar) : static_cast<double>(eq_t);
       mm = fmin(fmax(mm, 1.0), static_cast<double>(eq_t));
       const int k_thr = static_cast<int>(cab_t) + static_cast<int>(mm);
-      if (k_thr <= a.k_or_cap) {
+      if (k_thr <= kcap) {
         T = pf_t;
         cabove = cab_t;
         k_target = k_thr;
@@ -615,7 +643,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
     sel_before += gr + min(er, max(0, m_eq - eq_before));
     eq_before += er;
   }
-  int32_t* out = a.idx + (int64_t)h * a.ld_idx;
+  int32_t* out = a.idx + (int64_t)row_id * a.ld_idx;
   int pos = sel_before + G + min(E, max(0, m_eq - eq_before));
   int eq_seen = eq_before + E;
   for (int base = wb; base < wend; base += 32) {
@@ -631,24 +659,29 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelArgs a) {
     eq_seen += __popc(me);
   }
   // pad [k, k_or_cap) with -1, split over the cluster
-  for (int64_t t = (int64_t)k_target + rank * nt + tid; t < a.k_or_cap; t += (int64_t)C * nt) out[t] = -1;
-  if (rank == 0 && tid == 0) a.count[h] = k_target;
+  for (int64_t t = (int64_t)k_target + rank * nt + tid; t < kcap; t += (int64_t)C * nt) out[t] = -1;
+  if (rank == 0 && tid == 0) a.count[row_id] = k_target;
   cl.sync();  // keep shared memory alive until every remote read is done
 }
 
 cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mode, int k_or_cap,
                           double tau, double ln_alpha, int32_t* idx, int64_t ld_idx, int32_t* count, int* status,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const int32_t* cu, int64_t total, const int32_t* caps,
+                          int B) {
+  const int H_seq = H;  // heads of one sequence
+  H *= B;               // score rows of the launch
   int C = (N + 4095) / 4096;
   C = C < 1 ? 1 : (C > kSelMaxCluster ? kSelMaxCluster : C);
   {
-    // Many heads: a cluster per head at this size needs more than one wave of
-    // SMs (one CTA per SM).  The smallest cluster whose CTAs still cache their
-    // slice of the keys may fit all heads in one wave; take it then.
+    // Many rows: a cluster per row at this size needs more than one wave of
+    // SMs (one CTA per SM).  Then take the smallest cluster whose CTAs still
+    // cache their slice of the keys: it may fit all rows in one wave, and
+    // where it does not (a batch of many sequences), fewer CTAs per row spend
+    // less on the per-pass cluster barriers.
     int cmin = (N + kSelCacheKeys - 1) / kSelCacheKeys;
     cmin = cmin < 1 ? 1 : cmin;
     const int sms = device_sm_count();
-    if (cmin < C && H * C > sms && H * cmin <= sms) C = cmin;
+    if (cmin < C && H * C > sms) C = cmin;
   }
   const size_t mass_bytes = mode == VS_SELECT_THRESHOLD ? sizeof(double) * (kSelThreads / 32) * 256 : 0;
   // Room for the threshold rule's candidate list: what is left of the
@@ -694,7 +727,8 @@ cudaError_t launch_select(const float* scores, int H, int N, int64_t ld, int mod
   const int chunk = (N + C - 1) / C;
   const bool cache = chunk <= kSelCacheKeys;
   const int list_cap = list_entries(chunk, cache);
-  SelArgs a{scores, N, ld, mode, k_or_cap, tau, ln_alpha, idx, ld_idx, count, status, chunk, list_cap};
+  SelArgs a{scores, N,     ld,       mode, k_or_cap, tau,   ln_alpha, idx,
+            ld_idx, count, status, chunk, list_cap, cu,  total,    caps, H_seq};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, H, 1);
   cfg.blockDim = dim3(kSelThreads, 1, 1);

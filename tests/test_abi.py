@@ -93,6 +93,39 @@ def test_select_host_validation():
     assert call(N=1 << 21, ld=1 << 21) == vs.VS_ERR_UNSUPPORTED
 
 
+def test_select_varlen_host_validation():
+    L = vs.lib()
+    ws = _fake(0x20000)
+    good = dict(scores=_fake(), total=1000, B=3, cu=_fake(0x30000), maxn=600, H=2, mode=1,
+                caps=_fake(0x40000), cap_max=64, tau=0.9, idx=_fake(), ld_idx=64, cnt=_fake(),
+                ws=ws, wsb=256)
+
+    def call(**kw):
+        a = dict(good)
+        a.update(kw)
+        return L.vs_select_varlen(a["scores"], a["total"], a["B"], a["cu"], a["maxn"], a["H"],
+                                  a["mode"], a["caps"], a["cap_max"], a["tau"], a["idx"],
+                                  a["ld_idx"], a["cnt"], a["ws"], a["wsb"], None)
+
+    assert vs.vs_select_workspace_size_varlen(3, 2, 600) >= 256
+    for bad in ("scores", "cu", "caps", "idx", "cnt"):
+        assert call(**{bad: None}) == vs.VS_ERR_INVALID_ARG, bad
+    assert call(B=0) == vs.VS_ERR_INVALID_ARG
+    assert call(H=0) == vs.VS_ERR_INVALID_ARG
+    assert call(B=40000, H=2) == vs.VS_ERR_INVALID_ARG  # more than 65535 rows
+    assert call(maxn=0) == vs.VS_ERR_INVALID_ARG
+    assert call(total=0) == vs.VS_ERR_INVALID_ARG
+    assert call(cap_max=0) == vs.VS_ERR_INVALID_ARG
+    assert call(ld_idx=63) == vs.VS_ERR_INVALID_ARG
+    assert call(mode=7) == vs.VS_ERR_INVALID_ARG
+    assert call(tau=0.0) == vs.VS_ERR_INVALID_ARG
+    assert call(mode=2, tau=1.5) == vs.VS_ERR_INVALID_ARG
+    assert call(ws=None) == vs.VS_ERR_WORKSPACE
+    assert call(wsb=16) == vs.VS_ERR_WORKSPACE
+    assert call(ws=_fake(0x20010)) == vs.VS_ERR_WORKSPACE
+    assert call(maxn=(1 << 20) + 1) == vs.VS_ERR_UNSUPPORTED
+
+
 def test_attention_host_validation():
     L = vs.lib()
     f = _fake

@@ -139,8 +139,9 @@ def test_malformed_offsets_are_flagged_and_contained(cuda_device):
 
 @pytest.mark.slow
 def test_full_size_batch_workload(cuda_device):
-    # the bench's batch pipeline: per-sequence selects then one batched call;
-    # selections bit-exact against the oracle, rows of every sequence sampled
+    # the bench's batch pipeline: one batched select per score type, then one
+    # batched attention call; selections bit-exact against the oracle, rows of
+    # every sequence sampled
     from vs_testutil import sample_rows
     from vs_workloads import BATCH_WORKLOADS
     w = BATCH_WORKLOADS["llama_varlen_mix"]
@@ -148,21 +149,18 @@ def test_full_size_batch_workload(cuda_device):
     Q, K, V = (bf16_to_dev(x) for x in (Qb, Kb, Vb))
     B, H_sel, Hq = len(w.lengths), w.H_sel, w.Hq
     cu = w.cu_seqlens
+    cu_t = torch.from_numpy(cu).cuda()
     cap_max = w.cap(max(w.lengths))
-    vi = torch.full((B * H_sel, cap_max), -1, dtype=torch.int32, device="cuda")
-    si = torch.full_like(vi, -1)
-    vc = torch.empty(B * H_sel, dtype=torch.int32, device="cuda")
-    sc = torch.empty_like(vc)
+    caps = torch.tensor([w.cap(n) for n in w.lengths], dtype=torch.int32, device="cuda")
+    scores = [w.scores(b) for b in range(B)]
+    LV = torch.from_numpy(np.ascontiguousarray(np.concatenate([x[0] for x in scores], 1))).cuda()
+    LS = torch.from_numpy(np.ascontiguousarray(np.concatenate([x[1] for x in scores], 1))).cuda()
+    vi, vc = vs.select_varlen(LV, cu_t, max(w.lengths), w.select_mode_id, caps, cap_max, w.tau_v)
+    si, sc = vs.select_varlen(LS, cu_t, max(w.lengths), w.select_mode_id, caps, cap_max, w.tau_s)
     oracle_sets = []
     for b, n in enumerate(w.lengths):
-        lv, ls = w.scores(b)
+        lv, ls = scores[b]
         k = w.cap(n)
-        rows = slice(b * H_sel, (b + 1) * H_sel)
-        ws = vs.workspace(vs.vs_select_workspace_size(H_sel, n))
-        vs.vs_select(torch.from_numpy(lv).cuda(), w.select_mode_id, k, w.tau_v, vi[rows], vc[rows],
-                     ws)
-        vs.vs_select(torch.from_numpy(ls).cuda(), w.select_mode_id, k, w.tau_s, si[rows], sc[rows],
-                     ws)
         ovi, ovc, mv = oracle.select_heads(lv, w.select_mode_id, k, w.tau_v)
         osi, osc, ms = oracle.select_heads(ls, w.select_mode_id, k, w.tau_s)
         assert (mv >= 1e-9).all() and (ms >= 1e-9).all()
@@ -171,8 +169,7 @@ def test_full_size_batch_workload(cuda_device):
     ws = vs.workspace(vs.vs_attn_workspace_size_varlen(B, max_n, H_sel, w.d, cap_max))
     O = torch.empty_like(Q)
     lse = torch.empty((Hq, Q.shape[0]), dtype=torch.float32, device="cuda")
-    vs.vs_sparse_attn_fwd_varlen(Q, K, V, torch.from_numpy(cu).cuda(), max_n, vi, vc, si, sc, O,
-                                 lse, ws)
+    vs.vs_sparse_attn_fwd_varlen(Q, K, V, cu_t, max_n, vi, vc, si, sc, O, lse, ws)
     rc, flags = vs.vs_read_device_status(ws)
     assert rc == vs.VS_OK and flags == 0
     gvi, gvc, gsi, gsc = (x.cpu().numpy() for x in (vi, vc, si, sc))
