@@ -362,6 +362,33 @@ def ncu_traffic(workload: str):
 # --------------------------------------------------------------- our arm
 
 
+def vs_config(w, world: int, sharded: bool = False) -> dict:
+    """The `config` object of a vertical-slash workload's line (both arms)."""
+    return {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "H_sel": w.H_sel,
+            "select": w.select_mode, "k_v": w.k_v, "k_s": w.k_s, "tau_v": w.tau_v,
+            "tau_s": w.tau_s, "indexer": w.indexer,
+            "parallelism": f"heads x{world}" if sharded else f"replicas x{world}",
+            "l2": "inputs exceed L2 (Q/K/V/O resident in HBM) and a 256 MiB buffer is "
+                  "written between timed steps, outside the timed windows"}
+
+
+def batch_config(w, world: int) -> dict:
+    """The `config` object of a batch workload's line (both arms)."""
+    return {"workload": w.name, "sequences": len(w.lengths), "tokens": int(w.cu_seqlens[-1]),
+            "lengths": list(w.lengths), "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "H_sel": w.H_sel,
+            "select": w.select_mode, "cap_frac": w.cap_frac, "tau_v": w.tau_v, "tau_s": w.tau_s,
+            "parallelism": f"replicas x{world}",
+            "l2": "a 256 MiB buffer is written between timed steps, outside the timed windows"}
+
+
+def block_config(w, world: int) -> dict:
+    """The `config` object of a block-sparse workload's line (both arms)."""
+    return {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "alpha": w.alpha,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs exceed L2; a 256 MiB buffer is written between timed steps, "
+                  "outside the timed windows"}
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -679,12 +706,7 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
         "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded generators shaped like the pages' workloads)",
-        "config": {"workload": w.name, "N": N, "Hq": w.Hq, "Hkv": w.Hkv, "d": d, "H_sel": w.H_sel,
-                   "select": w.select_mode, "k_v": w.k_v, "k_s": w.k_s, "tau_v": w.tau_v,
-                   "tau_s": w.tau_s, "indexer": w.indexer,
-                   "parallelism": f"heads x{world}" if sharded else f"replicas x{world}",
-                   "l2": "inputs exceed L2 (Q/K/V/O resident in HBM) and a 256 MiB buffer is "
-                         "written between timed steps, outside the timed windows"},
+        "config": vs_config(w, world, sharded),
         "ms_per_layer": round(ms_step, 3), "ms_indexer": round(ms_idx, 3) if w.indexer else None,
         "ms_indexer_back_to_back": round(ms_idx_kernel, 3) if w.indexer else None,
         "ms_select": round(ms_sel, 3), "ms_attention": round(ms_att, 3),
@@ -866,7 +888,7 @@ def run_reference(args, w):
            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
            "data": "synthetic (seeded generators shaped like the pages' workloads)",
-           "config": {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d},
+           "config": vs_config(w, world),
            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"],
                             "kind": "oracle", "sample": last["sample"] + f"; {per_step:.1f} s per step"},
            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -939,8 +961,7 @@ def run_batch_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "impl": "reference",
         "data": "synthetic (seeded generators shaped like the pages' workloads)",
-        "config": {"workload": w.name, "sequences": B, "tokens": int(w.cu_seqlens[-1]),
-                   "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d},
+        "config": batch_config(w, world),
         "cpu_baseline": dict(last, value=round(value, 6),
                              sample=last["sample"] + f"; {per_step:.1f} s per step"),
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -1156,12 +1177,7 @@ def run_batch(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generators shaped like the pages' workloads)",
-        "config": {"workload": w.name, "sequences": B, "tokens": int(T), "lengths": list(w.lengths),
-                   "Hq": Hq, "Hkv": w.Hkv, "d": d, "H_sel": H_sel, "select": w.select_mode,
-                   "cap_frac": w.cap_frac, "tau_v": w.tau_v, "tau_s": w.tau_s,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "a 256 MiB buffer is written between timed steps, outside the timed "
-                         "windows"},
+        "config": batch_config(w, world),
         "ms_select": round(ms_step - ms_att, 3), "ms_attention": round(ms_att, 3),
         "selected_pairs": int(pairs), "density_vs_causal": round(pairs / dense_pairs, 5),
         "dense_ms": None if dense_ms is None else round(dense_ms, 3),
@@ -1370,10 +1386,7 @@ def run_blocks(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generators shaped like the pages' workloads)",
-        "config": {"workload": w.name, "N": N, "Hq": Hq, "Hkv": w.Hkv, "d": d, "alpha": w.alpha,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs exceed L2; a 256 MiB buffer is written between timed steps, "
-                         "outside the timed windows"},
+        "config": block_config(w, world),
         "ms_select": round(ms_step - ms_att, 3), "ms_attention": round(ms_att, 3),
         "selected_pairs": int(pairs), "density_vs_causal": round(pairs / dense_pairs, 5),
         "dense_ms": None if dense_ms is None else round(dense_ms, 3),
@@ -1475,8 +1488,7 @@ def run_blocks_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "impl": "reference",
         "data": "synthetic (seeded generators shaped like the pages' workloads)",
-        "config": {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "alpha": w.alpha},
+        "config": block_config(w, world),
         "cpu_baseline": dict(last, value=round(value, 6),
                              sample=last["sample"] + f"; {per_step:.1f} s per step"),
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
