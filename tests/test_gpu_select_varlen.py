@@ -143,3 +143,18 @@ def test_full_size_batch_workload_scores(cuda_device):
         idx, cnt, rc, flags = _run(packed, cu, caps, w.select_mode_id, tau, cap_max)
         assert rc == vs.VS_OK and flags == 0
         assert _check_rows(list(seqs), idx, cnt, caps, w.select_mode_id, tau) == []
+
+
+def test_many_long_rows_two_cta_clusters(cuda_device):
+    # rows longer than one CTA's key cache (32768 keys) and more rows than a
+    # wave of SMs holds at 8 CTAs per row: the launch takes 2-CTA clusters
+    rng = np.random.default_rng(8)
+    H = 4
+    lengths = tuple(int(x) for x in rng.integers(30000, 40001, 20))
+    seqs = [(rng.standard_normal((H, n)) * 2).astype(np.float32) for n in lengths]
+    caps = [n // 8 for n in lengths]
+    packed, cu = _pack(seqs)
+    for mode, tau in ((THR, 0.9), (TOPK, 1.0)):
+        idx, cnt, rc, flags = _run(packed, cu, caps, mode, tau, max(caps))
+        assert rc == vs.VS_OK and flags == 0
+        assert _check_rows(seqs, idx, cnt, caps, mode, tau) == []
