@@ -1009,6 +1009,7 @@ def run_batch(args, w):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     ev = {k: [] for k in ("s0", "a0", "a1")}
 
+    # a step launches 5 kernels: two batched selects, then plan, pack and attention
     def step(record):
         if record:
             e = torch.cuda.Event(enable_timing=True)
@@ -1186,7 +1187,7 @@ def run_batch(args, w):
                      "peak": peak, "unit": "TFLOP/s", "frac": round(t_roof_ms / ms_att, 4),
                      "traffic": None, "kernel": "vs_sparse_attn_fwd_varlen (plan + pack + attn)",
                      "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)"},
-        "e2e": e2e, "gpu_launches": (2 * B + 3) * args.steps, "input_gen_s": round(gen_s, 1),
+        "e2e": e2e, "gpu_launches": 5 * args.steps, "input_gen_s": round(gen_s, 1),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = batch_oracle_sample(w, Qb, Kb, Vb, (vih, vch, sih, sch),
